@@ -1,0 +1,179 @@
+/* looped.h - C ABI of the B200 (sm_100a) looped weight-shared decoder.
+ *
+ * The method: a decoder of 32 stored layers whose block of layers 4-27 runs
+ * twice with shared weights, B(B(h)), between a prelude (layers 0-3) and a
+ * coda (layers 28-31, then the output head): 4 + 24 + 24 + 4 = 56 layer
+ * executions per forward pass ("How Does SenseNova-Loop Get More Depth Without
+ * More Parameters?", section "What is the looped decoder in SenseNova-Loop?").
+ * Inside the block two residual streams are joined by manifold-constrained
+ * hyper-connections whose read, mix and write maps are learned, the mix being
+ * projected by 20 Sinkhorn row/column normalisations (same page, section
+ * "What does two-stream mHC do?").  Each 4-layer group is 3 linear-attention
+ * layers then 1 full-attention layer (same page, section "How does the hybrid
+ * attention pattern work?").  Shapes: hidden 4096, FFN 12288, vocabulary
+ * 248,320, contexts to 262,144 ("SenseTime's SenseNova-Loop-9B Runs Its Own
+ * Layers Twice, and It's Open Source", key-specs table).
+ *
+ * Conventions for every call:
+ *   - Status: 0 (LOOP_OK) or a negative LOOP_E* code; nothing is launched
+ *     when a call fails its argument checks.  loop_last_error() gives a text.
+ *   - Pointers named d_* are device pointers owned by the caller; they must
+ *     stay valid until the work queued on `stream` has finished.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous on that stream; one model must not
+ *     be used from two streams at once.
+ *   - The model owns its weights, its KV cache / linear-attention state arena
+ *     and its workspaces (device memory allocated by loop_model_create and
+ *     released by loop_model_destroy).
+ */
+#ifndef LOOPED_H
+#define LOOPED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LOOP_API __attribute__((visibility("default")))
+#else
+#define LOOP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  LOOP_OK = 0,
+  LOOP_EINVAL = -1,       /* bad argument or configuration                    */
+  LOOP_ENOMEM = -2,       /* device allocation failed (nothing is leaked)      */
+  LOOP_ECUDA = -3,        /* a CUDA call failed                                */
+  LOOP_ERANGE = -4,       /* batch > max_batch or context > max_ctx            */
+  LOOP_EUNSUPPORTED = -5, /* valid configuration this build does not run       */
+  LOOP_ETIMEOUT = -6      /* a device-side wait gave up (see loop_device_status) */
+};
+
+enum { LOOP_F32 = 0, LOOP_BF16 = 1 };
+enum { LOOP_TOKENS_TO_LOGITS = 0, LOOP_HIDDEN_TO_HIDDEN = 1 };
+enum { LOOP_ALL_POSITIONS = 1u }; /* loop_prefill flag: logits for every position */
+enum { LOOP_KIND_LINEAR = 0, LOOP_KIND_FULL = 1 };
+enum { LOOP_REGION_PRELUDE = 0, LOOP_REGION_BLOCK = 1, LOOP_REGION_CODA = 2 };
+
+/* The checkpoint's execution configuration: loop range, pass count and mHC
+ * settings travel with the weights, because a plain layer-by-layer runner
+ * would execute the wrong order ("How Does SenseNova-Loop Get More Depth
+ * Without More Parameters?", section "How do you run SenseNova-Loop-9B-Preview?").
+ * The loop-9B values are given in brackets. */
+typedef struct {
+  int32_t n_prelude, n_block, n_loops, n_coda; /* [4, 24, 2, 4]; n_prelude, n_block multiples of group */
+  int32_t group, full_slot;                    /* [4, 3]: layer p is full attention iff p % group == full_slot */
+  int32_t hidden, ffn, vocab;                  /* [4096, 12288, 248320]; vocab unused for HIDDEN_TO_HIDDEN */
+  int32_t n_q, n_kv, head_dim;                 /* full attention, GQA [32, 8, 128] */
+  int32_t n_lin, lin_dim, lin_chunk;           /* gated linear attention [32, 128, 64] */
+  int32_t n_streams, sinkhorn_iters;           /* mHC [2, 20]; this build runs n_streams == 2 */
+  float rope_base, norm_eps;                   /* [1e4, 1e-6] */
+  int32_t dtype;                               /* LOOP_F32 or LOOP_BF16 (mHC parameters are always fp32) */
+  int32_t io_mode;                             /* LOOP_TOKENS_TO_LOGITS or LOOP_HIDDEN_TO_HIDDEN */
+  int32_t max_batch, max_ctx;                  /* size of the cache arena */
+} loop_config;
+
+typedef struct loop_model loop_model;
+
+/* Number of layer executions n_prelude + n_block * n_loops + n_coda, or a
+ * negative status for an invalid configuration. */
+LOOP_API int32_t loop_num_exec(const loop_config* cfg);
+
+/* Execution table (host memory, 5 int32 per execution): physical layer,
+ * pass, kind (LOOP_KIND_*), cache slot, region (LOOP_REGION_*).  Prelude
+ * execution e runs layer e; block execution n_prelude + p * n_block + j runs
+ * layer n_prelude + j in pass p (B(B(h))); the coda runs the remaining layers.
+ * The k-th full-attention execution owns KV slot k and the k-th linear one
+ * owns state slot k, so each pass keeps its own caches.  Returns the number of
+ * executions or a negative status. */
+LOOP_API int32_t loop_schedule(const loop_config* cfg, int32_t* table);
+
+/* Number of weight tensors in the canonical order used by loop_model_create:
+ * [0] embedding [vocab][hidden] (empty for HIDDEN_TO_HIDDEN), [1] final norm
+ * gain [hidden]; then per physical layer 10 tensors: attention-norm gain, W_q,
+ * W_k, W_v, W_g (linear layers only; empty for full attention), W_o, FFN-norm
+ * gain, W_gate, W_up, W_down (matrices stored [out][in]); then per block layer
+ * and sublayer (attention, FFN) the mHC gain gamma [n*hidden] and projection
+ * Phi [2n + n*n][n*hidden].  Negative status for an invalid configuration. */
+LOOP_API int32_t loop_num_weights(const loop_config* cfg);
+
+/* Create a model.  host_weights == NULL draws every matrix from the seeded
+ * SplitMix64 generator on the device (0.02 * N(0,1), rounded to the model
+ * dtype; norm gains 1); otherwise host_weights[i] points to host fp32 values of
+ * tensor i in the canonical order above (copied and converted; the caller
+ * keeps ownership).  Allocates the weights, the per-execution KV cache and
+ * linear-attention state for max_batch x max_ctx, and the workspaces.  Blocks
+ * until the model is ready.  On failure *out is NULL and nothing is leaked. */
+LOOP_API int32_t loop_model_create(const loop_config* cfg, const float* const* host_weights, uint64_t seed,
+                          loop_model** out);
+
+/* Prefill B sequences of S tokens from position 0 (resets their caches).
+ * TOKENS_TO_LOGITS: d_tokens int32 [B][S] (each in [0, vocab)); d_out fp32
+ *   [B][vocab] with the logits of each sequence's last position, or
+ *   [B][S][vocab] when flags has LOOP_ALL_POSITIONS.
+ * HIDDEN_TO_HIDDEN: d_hidden fp32 [B][S][hidden] in, d_out fp32 [B][S][hidden]
+ *   out (the collapsed streams; no embedding, final norm or head).
+ * Writes each execution's KV (positions 0..S-1) and final linear-attention
+ * state into its own slot; afterwards the sequences have length S.
+ * LOOP_ERANGE if B > max_batch or S > max_ctx. */
+LOOP_API int32_t loop_prefill(loop_model* m, const int32_t* d_tokens, const float* d_hidden, int32_t B, int32_t S,
+                     float* d_out, uint32_t flags, void* stream);
+
+/* One decode step for sequences 0..B-1: d_tokens int32 [B] is the next token
+ * of each sequence, processed at its current length; d_logits fp32 [B][vocab].
+ * Appends one KV position per full-attention execution, advances every
+ * linear-attention state, then adds 1 to each sequence length.
+ * LOOP_ERANGE if a sequence would pass max_ctx. */
+LOOP_API int32_t loop_decode_step(loop_model* m, const int32_t* d_tokens, int32_t B, float* d_logits, void* stream);
+
+/* Sinkhorn projection of `count` n x n matrices (fp32, row-major, device):
+ * P = exp(L - max L) with the library's fixed exponential (Cody-Waite
+ * reduction and a degree-7 Taylor polynomial, fused multiply-adds), then
+ * `iters` times: divide each row by its sum, then each column by its sum
+ * (sums left to right, IEEE division).  The result is bit-identical across
+ * runs and to any implementation of that same definition.  The mixing map of
+ * the mHC streams ("How Does SenseNova-Loop Get More Depth Without More
+ * Parameters?", section "What does two-stream mHC do?").  n in [1, 8]. */
+LOOP_API int32_t mhc_sinkhorn(const float* d_logits, float* d_out, int32_t count, int32_t n, int32_t iters, void* stream);
+
+/* Release everything the model owns.  Waits for the model's queued work. */
+LOOP_API void loop_model_destroy(loop_model* m);
+
+/* ---- inspection (tests and tools) ---- */
+
+/* Current length of sequence b (host value kept in step with the device). */
+LOOP_API int32_t loop_seq_len(const loop_model* m, int32_t b);
+
+/* Copy a cache slot to d_out (device, fp32): kind LOOP_KIND_FULL gives K then
+ * V, each [B][n_kv][len][head_dim]; LOOP_KIND_LINEAR gives the state
+ * [B][n_lin][lin_dim][lin_dim] (S[k][v]). */
+LOOP_API int32_t loop_cache_read(loop_model* m, int32_t kind, int32_t slot, int32_t B, int32_t len, float* d_out,
+                        void* stream);
+
+/* Copy weight tensor `index` (canonical order, see loop_num_weights) to d_out
+ * (device, fp32) in its canonical row-major [out][in] layout. */
+LOOP_API int32_t loop_weight_read(loop_model* m, int32_t index, float* d_out, void* stream);
+
+/* The projection primitive on its own: C[M][N] (row stride ldc, fp32) =
+ * A[M][K] W[N][K]^T with A, W bf16 row-major device arrays.  use_tensor_cores
+ * selects the tcgen05 kernel (K a multiple of 64; LOOP_EUNSUPPORTED otherwise)
+ * or the CUDA-core kernel. */
+LOOP_API int32_t loop_gemm_bf16(const void* d_A, const void* d_W, int64_t M, int64_t N, int64_t K, float* d_C,
+                                int64_t ldc, int32_t use_tensor_cores, void* stream);
+
+/* Sticky device status word: 0, or the bits of waits that timed out in a
+ * kernel (the kernel then returned early).  Reading it synchronises the
+ * device.  loop_clear_device_status() resets it. */
+LOOP_API int32_t loop_device_status(void);
+LOOP_API void loop_clear_device_status(void);
+
+/* Text of the last failed call on this thread ("" if none). */
+LOOP_API const char* loop_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

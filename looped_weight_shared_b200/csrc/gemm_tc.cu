@@ -1,0 +1,465 @@
+// Tensor-core projection GEMM for sm_100a: C = A[M][K] W[N][K]^T in bf16 with
+// fp32 accumulation in tensor memory, followed by the projection's epilogue
+// (residual add, mHC stream write, SwiGLU, q/k/v split with L2 norm or RoPE
+// and KV-cache write, or plain fp32 logits).
+//
+// Persistent kernel, one CTA per SM, warp-specialised:
+//   warp 0      TMA producer: A tile 128 x 64 and W tile 256 x 64 per stage,
+//               128-byte swizzle, 4 stages in shared memory;
+//   warp 1      one thread issues tcgen05.mma (M = 128, N = 256, K = 16) into
+//               one of two 256-column TMEM accumulators;
+//   warp 2      allocates / frees the 512 TMEM columns;
+//   warps 4-7   epilogue: tcgen05.ld of the accumulator rows (warp w reads
+//               TMEM lanes 32 (w % 4) ..), fused output, then release the
+//               accumulator so the next tile's MMAs overlap this epilogue.
+// Every wait on an mbarrier gives up after ~2 s and flags the status word.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "model.h"
+
+namespace loopk {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int THREADS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int GROUP_M = 16;  // tile raster: GROUP_M row blocks sweep the N blocks together
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+struct EpiP {
+  int M, N;
+  float* c;
+  int64_t ldc;
+  float* s;
+  const float* coef;
+  bf16* a;
+  bf16* q;
+  bf16* k;
+  bf16* v;
+  float* gl;
+  const float2* rope;
+  const int32_t* start;
+  int S, hq, hkv, n_lin;
+  int64_t ctx;
+  float eps;
+};
+
+LOOP_DEV void ld_chunk(uint32_t taddr, float (&v)[32]) {
+  tmem_ld32(taddr, v);
+  tc_wait_ld();
+}
+
+LOOP_DEV void store_bf16x32(bf16* dst, const float (&v)[32], float scale) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 u;
+    u.x = pack_bf16x2(v[8 * i + 0] * scale, v[8 * i + 1] * scale);
+    u.y = pack_bf16x2(v[8 * i + 2] * scale, v[8 * i + 3] * scale);
+    u.z = pack_bf16x2(v[8 * i + 4] * scale, v[8 * i + 5] * scale);
+    u.w = pack_bf16x2(v[8 * i + 6] * scale, v[8 * i + 7] * scale);
+    d[i] = u;
+  }
+}
+
+// L2-normalise (optional) one 128-column head held in TMEM and store it bf16.
+// Every lane runs the TMEM loads (warp-collective); only rows < M store.
+LOOP_DEV void head_store(uint32_t t0, bf16* dst, bool l2, float eps, bool valid) {
+  float scale = 1.f;
+  float v[32];
+  if (l2) {
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      ld_chunk(t0 + 32 * c, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ss += v[j] * v[j];
+    }
+    scale = rsqrtf(ss + eps);
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    ld_chunk(t0 + 32 * c, v);
+    if (valid) store_bf16x32(dst + 32 * c, v, scale);
+  }
+}
+
+// Rotate-half RoPE on one 128-column head held in TMEM, then store bf16.
+LOOP_DEV void head_store_rope(uint32_t t0, bf16* dst, const float2* cs_row, bool valid) {
+#pragma unroll 1
+  for (int c = 0; c < 2; ++c) {
+    float a[32], b[32];
+    ld_chunk(t0 + 32 * c, a);
+    ld_chunk(t0 + 64 + 32 * c, b);
+    if (!valid) continue;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float2 cs = cs_row[32 * c + j];
+      const float x = a[j], y = b[j];
+      a[j] = x * cs.x - y * cs.y;
+      b[j] = y * cs.x + x * cs.y;
+    }
+    store_bf16x32(dst + 32 * c, a, 1.f);
+    store_bf16x32(dst + 64 + 32 * c, b, 1.f);
+  }
+}
+
+// tcgen05.ld / wait::ld are warp-collective: every lane of the warp executes
+// them in lockstep, and only the memory accesses of rows >= M are skipped.
+template <Epi MODE>
+LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, const EpiP& p) {
+  const bool valid = row < p.M;
+  if constexpr (MODE == Epi::F32) {
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int n = n0 + 32 * c;
+      if (n >= p.N) break;
+      float v[32];
+      ld_chunk(tacc + 32 * c, v);
+      if (!valid) continue;
+      float* dst = p.c + (int64_t)row * p.ldc + n;
+      if (n + 32 <= p.N && (p.ldc % 4) == 0) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          reinterpret_cast<float4*>(dst)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      } else {
+        for (int j = 0; j < 32 && n + j < p.N; ++j) dst[j] = v[j];
+      }
+    }
+  } else if constexpr (MODE == Epi::RESID) {
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int n = n0 + 32 * c;
+      float v[32];
+      ld_chunk(tacc + 32 * c, v);
+      if (!valid) continue;
+      float4* h = reinterpret_cast<float4*>(p.c + (int64_t)row * p.N + n);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 x = h[j];
+        x.x += v[4 * j]; x.y += v[4 * j + 1]; x.z += v[4 * j + 2]; x.w += v[4 * j + 3];
+        h[j] = x;
+      }
+    }
+  } else if constexpr (MODE == Epi::MHC_WRITE) {
+    const int crow = valid ? row : 0;
+    const float4 c0 = reinterpret_cast<const float4*>(p.coef + (int64_t)crow * 8)[0];
+    const float4 c1 = reinterpret_cast<const float4*>(p.coef + (int64_t)crow * 8)[1];
+    // c0 = (pre0, pre1, post0, post1), c1 = (res00, res01, res10, res11)
+    const int64_t plane = (int64_t)p.M * p.N;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int n = n0 + 32 * c;
+      float v[32];
+      ld_chunk(tacc + 32 * c, v);
+      if (!valid) continue;
+      float4* s0 = reinterpret_cast<float4*>(p.s + (int64_t)row * p.N + n);
+      float4* s1 = reinterpret_cast<float4*>(p.s + plane + (int64_t)row * p.N + n);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 a = s0[j], b = s1[j];
+        float4 x, y;
+        x.x = c1.x * a.x + c1.y * b.x + c0.z * v[4 * j + 0];
+        x.y = c1.x * a.y + c1.y * b.y + c0.z * v[4 * j + 1];
+        x.z = c1.x * a.z + c1.y * b.z + c0.z * v[4 * j + 2];
+        x.w = c1.x * a.w + c1.y * b.w + c0.z * v[4 * j + 3];
+        y.x = c1.z * a.x + c1.w * b.x + c0.w * v[4 * j + 0];
+        y.y = c1.z * a.y + c1.w * b.y + c0.w * v[4 * j + 1];
+        y.z = c1.z * a.z + c1.w * b.z + c0.w * v[4 * j + 2];
+        y.w = c1.z * a.w + c1.w * b.w + c0.w * v[4 * j + 3];
+        s0[j] = x;
+        s1[j] = y;
+      }
+    }
+  } else if constexpr (MODE == Epi::SWIGLU) {
+    const int F = p.N / 2;
+    bf16* dst = p.a + (int64_t)row * F + n0 / 2;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float g[32], u[32];
+      ld_chunk(tacc + 32 * c, g);
+      ld_chunk(tacc + 128 + 32 * c, u);
+      if (!valid) continue;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) g[j] = g[j] / (1.f + __expf(-g[j])) * u[j];
+      store_bf16x32(dst + 32 * c, g, 1.f);
+    }
+  } else if constexpr (MODE == Epi::QKV_LINEAR) {
+    const int d = 128, nl = p.n_lin;
+    const int b = row / p.S, t = row % p.S;
+    const int region = n0 / (nl * d);  // 0 q, 1 k, 2 v, 3 gate
+    if (region < 3) {
+      bf16* base = region == 0 ? p.q : (region == 1 ? p.k : p.v);
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        const int head = (n0 - region * nl * d) / d + hh;
+        bf16* dst = base + (((int64_t)b * nl + head) * p.S + t) * d;
+        head_store(tacc + 128 * hh, dst, region < 2, p.eps, valid);
+      }
+    } else {
+      float v[32];
+#pragma unroll 1
+      for (int c = 0; c * 32 < nl; ++c) {
+        ld_chunk(tacc + 32 * c, v);
+        if (!valid) continue;
+        for (int j = 0; j < 32 && 32 * c + j < nl; ++j) {
+          const int head = 32 * c + j;
+          const float z = v[j];
+          p.gl[((int64_t)b * nl + head) * p.S + t] = z >= 0.f ? -log1pf(__expf(-z)) : z - log1pf(__expf(z));
+        }
+      }
+    }
+  } else if constexpr (MODE == Epi::QKV_FULL) {
+    const int d = 128;
+    const int b = row / p.S, t = row % p.S;
+    const int64_t pos = valid ? p.start[b] + t : 0;
+    const float2* cs = p.rope + pos * (d / 2);
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+      const int head = n0 / d + hh;
+      const uint32_t t0 = tacc + 128 * hh;
+      if (head < p.hq) {
+        head_store_rope(t0, p.q + (((int64_t)b * p.hq + head) * p.S + t) * d, cs, valid);
+      } else if (head < p.hq + p.hkv) {
+        head_store_rope(t0, p.k + (((int64_t)b * p.hkv + (head - p.hq)) * p.ctx + pos) * d, cs, valid);
+      } else {
+        head_store(t0, p.v + (((int64_t)b * p.hkv + (head - p.hq - p.hkv)) * p.ctx + pos) * d, false, 0.f,
+                   valid);
+      }
+    }
+  }
+}
+
+LOOP_DEV void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
+  const int per_group = GROUP_M * num_n;
+  const int g = tile / per_group;
+  const int first = g * GROUP_M;
+  const int gsz = min(num_m - first, GROUP_M);
+  const int r = tile % per_group;
+  mb = first + r % gsz;
+  nb = r / gsz;
+}
+
+template <Epi MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb, int M, int N,
+                   int K, EpiP p, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sa = smem;
+  uint8_t* sb = smem + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN, tiles = num_m * num_n;
+  const int kbs = K / BK;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tma);
+    prefetch_tmap(&tmb);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, mb, nb);
+      for (int kb = 0; kb < kbs; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, status, STATUS_WAIT_PRODUCER)) { ok = false; break; }
+        mbar_expect_tx(&full[stage], STAGE_BYTES);
+        tma_load_2d(sa + stage * A_BYTES, &tma, &full[stage], kb * BK, mb * BM);
+        tma_load_2d(sb + stage * B_BYTES, &tmb, &full[stage], kb * BK, nb * BN);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    int stage = 0;
+    uint32_t phase = 0;
+    int local = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t aphase = (local >> 1) & 1;
+      if (!mbar_wait(&tempty[acc], aphase ^ 1, status, STATUS_WAIT_MMA)) break;
+      tc_fence_after();
+      const uint32_t d = tmem + acc * BN;
+      for (int kb = 0; kb < kbs; ++kb) {
+        if (!mbar_wait(&full[stage], phase, status, STATUS_WAIT_MMA)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sa + stage * A_BYTES), b0 = smem_u32(sb + stage * B_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint64_t ad = smem_desc_sw128(a0 + 32 * k, 1024);
+          const uint64_t bd = smem_desc_sw128(b0 + 32 * k, 1024);
+          tc_mma_f16(d, ad, bd, IDESC, (kb | k) != 0);
+        }
+        tc_commit(&empty[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (ok) tc_commit(&tfull[acc]);
+    }
+  } else if (warp >= 4) {
+    const int q = warp & 3;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t aphase = (local >> 1) & 1;
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, mb, nb);
+      const bool got = mbar_wait(&tfull[acc], aphase, status, STATUS_WAIT_EPILOGUE);
+      if (!__all_sync(0xffffffffu, got)) break;  // the whole warp leaves together
+      tc_fence_after();
+      const uint32_t tacc = tmem + acc * BN + ((uint32_t)(32 * q) << 16);
+      epilogue_tile<MODE>(tacc, mb * BM + 32 * q + lane, nb * BN, p);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows][K] matrix, box 64 x box_rows,
+// 128-byte swizzle; rows past the end read as zeros.
+bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <Epi MODE>
+cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K, const EpiP& p,
+                        cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = std::min(tiles, num_sms());
+  gemm_tc_kernel<MODE><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, M, N, K, p, status_ptr());
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc_supported(int64_t M, int64_t N, int64_t K, const EpiArgs& e) {
+  if (M <= 0 || K % BK != 0 || M > (int64_t)1 << 30 || N > (int64_t)1 << 30) return false;
+  switch (e.mode) {
+    case Epi::F32: return true;
+    case Epi::RESID:
+    case Epi::MHC_WRITE: return N % BN == 0;
+    case Epi::SWIGLU: return N % BN == 0;
+    case Epi::QKV_LINEAR: return e.hd == 128 && ((int64_t)e.n_lin * 128) % BN == 0 && e.n_lin <= BN;
+    case Epi::QKV_FULL: return e.hd == 128 && N % BN == 0 && ((int64_t)e.heads_q * 128) % BN == 0 &&
+                               ((int64_t)e.heads_kv * 128) % BN == 0;
+  }
+  return false;
+}
+
+cudaError_t launch_gemm_tc(const void* A, const void* W, int64_t M, int64_t N, int64_t K, const EpiArgs& e,
+                           cudaStream_t st) {
+  if (!gemm_tc_supported(M, N, K, e)) return cudaErrorNotSupported;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, M, K, BM) || !make_map(&mb, W, N, K, BN)) return cudaErrorInvalidValue;
+  EpiP p{};
+  p.M = (int)M;
+  p.N = (int)N;
+  p.c = e.c;
+  p.ldc = e.ldc;
+  p.s = e.s;
+  p.coef = e.coef;
+  p.a = (bf16*)e.a;
+  p.q = (bf16*)e.q;
+  p.k = (bf16*)e.k;
+  p.v = (bf16*)e.v;
+  p.gl = e.gl;
+  p.rope = e.rope;
+  p.start = e.start;
+  p.S = e.S;
+  p.hq = e.heads_q;
+  p.hkv = e.heads_kv;
+  p.n_lin = e.n_lin;
+  p.ctx = e.cache_ctx;
+  p.eps = e.eps;
+  switch (e.mode) {
+    case Epi::F32: return launch_mode<Epi::F32>(ma, mb, (int)M, (int)N, (int)K, p, st);
+    case Epi::RESID: return launch_mode<Epi::RESID>(ma, mb, (int)M, (int)N, (int)K, p, st);
+    case Epi::MHC_WRITE: return launch_mode<Epi::MHC_WRITE>(ma, mb, (int)M, (int)N, (int)K, p, st);
+    case Epi::SWIGLU: return launch_mode<Epi::SWIGLU>(ma, mb, (int)M, (int)N, (int)K, p, st);
+    case Epi::QKV_LINEAR: return launch_mode<Epi::QKV_LINEAR>(ma, mb, (int)M, (int)N, (int)K, p, st);
+    case Epi::QKV_FULL: return launch_mode<Epi::QKV_FULL>(ma, mb, (int)M, (int)N, (int)K, p, st);
+  }
+  return cudaErrorNotSupported;
+}
+
+}  // namespace loopk

@@ -1,0 +1,144 @@
+// Internal declarations of the looped-decoder library: the model object, its
+// workspace, and the launchers each kernel file provides.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/looped.h"
+#include "common.cuh"
+
+namespace loopk {
+
+// Output modes of a projection (a GEMM C = A W^T plus what follows it).
+enum class Epi {
+  F32,         // C fp32 [M][N] (row stride ldc) - logits
+  RESID,       // h[M][H] += C                     (prelude / coda residual)
+  MHC_WRITE,   // s_i = sum_j res[i][j] s_j + post[i] C   (two streams)
+  SWIGLU,      // a[M][F] = silu(C gate) * C up; weight rows interleaved per 128
+  QKV_LINEAR,  // q, k (L2-normalised), v -> [B][n_lin][S][d]; log sigmoid(gate) -> [B][n_lin][S]
+  QKV_FULL,    // RoPE(q) -> [B][n_q][S][hd]; RoPE(k), v -> cache [B][n_kv][max_ctx][hd]
+};
+
+struct EpiArgs {
+  Epi mode = Epi::F32;
+  float* c = nullptr;  // F32: output; RESID: h
+  int64_t ldc = 0;
+  float* s = nullptr;  // MHC_WRITE: streams [2][M][H]
+  const float* coef = nullptr;  // MHC_WRITE: [M][8]
+  void* a = nullptr;            // SWIGLU output [M][F]
+  void* q = nullptr;            // QKV: q [B][heads][S][d]
+  void* k = nullptr;            // QKV_LINEAR: k; QKV_FULL: K cache base (sequence b0)
+  void* v = nullptr;            // QKV_LINEAR: v; QKV_FULL: V cache base
+  float* gl = nullptr;          // QKV_LINEAR: log-gates [B][n_lin][S]
+  const float2* rope = nullptr; // QKV_FULL: (cos, sin) [max_ctx][hd/2]
+  const int32_t* start = nullptr;  // QKV_FULL: start position of each sequence
+  int S = 1;                    // tokens per sequence in this call
+  int heads_q = 0, heads_kv = 0, hd = 0;
+  int64_t cache_ctx = 0;        // QKV_FULL: max_ctx (position stride of the cache)
+  int n_lin = 0;
+  float eps = 1e-6f;
+};
+
+struct LayerW {
+  bool full = false;
+  void* w_in = nullptr;   // linear: [3 n_lin d + n_lin][H] (q | k | v | gate); full: [(n_q + 2 n_kv) hd][H]
+  void* w_o = nullptr;    // [H][n d]
+  void* w_gu = nullptr;   // [2F][H]: block j of 256 rows = gate rows 128j.. then up rows 128j..
+  void* w_down = nullptr; // [H][F]
+  float* attn_gain = nullptr;
+  float* ffn_gain = nullptr;
+  int64_t n_in = 0, n_o_in = 0;
+};
+
+struct SiteW {
+  float* gamma = nullptr;  // [2H]
+  float* phi = nullptr;    // [8][2H]
+};
+
+struct Work {
+  int64_t t_max = 0;
+  float* h = nullptr;       // [T][H]
+  float* s = nullptr;       // [2][T][H]
+  void* xh = nullptr;       // [T][H]
+  float* coef = nullptr;    // [T][8]
+  void* q = nullptr;        // [T][max(n_q hd, n_lin d)]
+  void* k = nullptr;        // [T][n_lin d]
+  void* v = nullptr;        // [T][n_lin d]
+  float* gl = nullptr;      // [T][n_lin]
+  void* o = nullptr;        // [T][max(n_q hd, n_lin d)]
+  void* a = nullptr;        // [T][F]
+  float* cbuf = nullptr;    // [T][max N] projection scratch of the unfused path
+  void* xf = nullptr;       // [rows][H] final-norm output
+  int32_t* zeros = nullptr; // start positions of a prefill (all 0)
+  float* gla_scratch = nullptr;
+  int64_t gla_scratch_floats = 0;
+};
+
+struct Model {
+  loop_config c{};
+  int n_phys = 0, n_exec = 0, n_full = 0, n_lin = 0;
+  std::vector<int32_t> table;
+  size_t esize = 4;
+  void* embed = nullptr;
+  float* final_gain = nullptr;
+  std::vector<LayerW> L;
+  std::vector<SiteW> sites;
+  std::vector<void*> kc, vc;    // per full-attention slot [max_batch][n_kv][max_ctx][hd]
+  std::vector<float*> st;       // per linear slot [max_batch][n_lin][d][d] fp32
+  int32_t* d_seq_len = nullptr;
+  std::vector<int32_t> seq_len;
+  float2* rope = nullptr;       // [max_ctx][hd/2]
+  Work w;
+  std::vector<void*> allocs;
+  bool use_tc = false;          // tcgen05 path for bf16 projections
+};
+
+bool bf16_model(const Model& m);
+
+// Device address of the library's status word (this device), or NULL.
+int* status_ptr();
+int status_read();
+void status_clear();
+
+// ---- launchers (each returns cudaGetLastError()) ----
+cudaError_t launch_fill_normal(void* dst, bool bf16, int64_t rows, int64_t cols, int64_t dst_row0,
+                               uint64_t seed, uint64_t stream, int64_t src_row0, double scale, cudaStream_t st);
+cudaError_t launch_fill_const(float* dst, int64_t n, float v, cudaStream_t st);
+cudaError_t launch_embed(const int32_t* tok, const void* E, bool bf16, int64_t T, int H, int V, float* h,
+                         cudaStream_t st);
+cudaError_t launch_rmsnorm(const float* x, int64_t rows, int H, int64_t row_step, int64_t row_off,
+                           const float* gain, float eps, void* y, bool bf16, cudaStream_t st);
+cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,
+                                const float* gain, int iters, float eps, float* coef, void* xh, bool bf16,
+                                cudaStream_t st);
+cudaError_t launch_expand(const float* h, float* s, int64_t n, cudaStream_t st);
+cudaError_t launch_collapse(const float* s, float* h, int64_t n, cudaStream_t st);
+cudaError_t launch_sinkhorn(const float* l, float* out, int64_t count, int n, int iters, cudaStream_t st);
+
+cudaError_t launch_gemm_simt(const void* A, const void* W, bool bf16, int64_t M, int64_t N, int64_t K,
+                             float* C, int64_t ldc, cudaStream_t st);
+cudaError_t launch_epilogue_unfused(const float* C, int64_t ldc, int64_t M, int64_t N, const EpiArgs& e, bool bf16,
+                                    cudaStream_t st);
+cudaError_t launch_attention_simple(const void* q, const void* K, const void* V, void* o, bool bf16, int B, int S,
+                                    int nq, int nkv, int hd, int64_t cache_ctx, const int32_t* start,
+                                    cudaStream_t st);
+cudaError_t launch_gla_recurrent(const void* q, const void* k, const void* v, const float* gl, float* state, void* o,
+                                 bool bf16, int B, int S, int nh, int d, cudaStream_t st);
+cudaError_t launch_rope_table(float2* tab, int64_t ctx, int hd, double base, cudaStream_t st);
+cudaError_t launch_cache_to_f32(const void* src, bool bf16, int B, int nkv, int64_t ctx, int len, int hd,
+                                float* dst, cudaStream_t st);
+cudaError_t launch_advance(int32_t* seq_len, int B, cudaStream_t st);
+cudaError_t launch_set_len(int32_t* seq_len, int B, int S, cudaStream_t st);
+cudaError_t launch_weight_to_f32(const void* src, bool bf16, int64_t rows, int64_t cols, int64_t src_row0,
+                                 float* dst, cudaStream_t st);
+
+// tcgen05 GEMM (bf16): C = A[M][K] W[N][K]^T with a fused epilogue.  Returns
+// cudaErrorNotSupported when the shapes are outside what it handles.
+cudaError_t launch_gemm_tc(const void* A, const void* W, int64_t M, int64_t N, int64_t K, const EpiArgs& e,
+                           cudaStream_t st);
+bool gemm_tc_supported(int64_t M, int64_t N, int64_t K, const EpiArgs& e);
+
+}  // namespace loopk

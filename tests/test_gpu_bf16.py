@@ -1,0 +1,76 @@
+"""GPU parity of the bf16 path against the oracle in its bf16 mode
+(tolerance: max-abs relative error 2e-2 and cosine >= 0.999)."""
+
+import numpy as np
+import pytest
+
+import oracle
+import seeded
+from seeded import workloads as W
+from metrics import COS_BF16, TOL_BF16, cosine, rel_err
+
+torch = pytest.importorskip("torch")
+import looped_weight_shared_b200 as L  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+def check(got, ref):
+    e, c = rel_err(got, ref), cosine(got, ref)
+    assert e < TOL_BF16 and c > COS_BF16, (e, c)
+    return e, c
+
+
+def test_tiny_bf16_prefill_and_decode():
+    m = dict(W.model_config("tiny_fp32", dtype=1), max_batch=3, max_ctx=200)
+    g = L.loop_model_create(L.make_config(**m), seed=0)
+    try:
+        o = oracle.Model(oracle.make_config(**m), seed=0)
+        tok = seeded.tokens(3, 3, 150, m["vocab"])
+        ref = o.prefill(tok, all_positions=True)
+        out = torch.empty((3, 150, m["vocab"]), device="cuda")
+        L.loop_prefill(g, tokens=torch.from_numpy(tok).cuda(), out=out, flags=L.LOOP_ALL_POSITIONS)
+        torch.cuda.synchronize()
+        check(out.cpu().numpy(), ref)
+        nxt = seeded.tokens(3, 3, 3, m["vocab"], stream=seeded.S_DECODE_TOKENS)
+        for t in range(3):
+            r = o.decode_step(nxt[:, t])
+            d = torch.empty((3, m["vocab"]), device="cuda")
+            L.loop_decode_step(g, torch.from_numpy(np.ascontiguousarray(nxt[:, t])).cuda(), d)
+            torch.cuda.synchronize()
+            check(d.cpu().numpy(), r)
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
+
+
+@pytest.mark.parametrize("S", [160])
+def test_group9b_bf16_matches_oracle(S):
+    """One 4-layer group at the 9B width (3 GLA + 1 full attention, hidden
+    4096, FFN 12288) run twice with shared weights, hidden in -> hidden out."""
+    m = dict(W.model_config("group9b_s4096"), max_batch=1, max_ctx=S)
+    g = L.loop_model_create(L.make_config(**m), seed=1)
+    try:
+        o = oracle.Model(oracle.make_config(**m), seed=1)
+        h = seeded.hidden(1, 1, S, m["hidden"])
+        ref = o.prefill(hidden=h)
+        out = torch.empty((1, S, m["hidden"]), device="cuda")
+        L.loop_prefill(g, hidden=torch.from_numpy(h).cuda(), out=out)
+        torch.cuda.synchronize()
+        check(out.cpu().numpy(), ref)
+        # the states and caches of both passes
+        for slot in range(6):
+            st = torch.empty((1, 32, 128, 128), device="cuda")
+            L.loop_cache_read(g, L.LOOP_KIND_LINEAR, slot, 1, 0, st)
+            torch.cuda.synchronize()
+            check(st.cpu().numpy(), o.state(slot, 1))
+        for slot in range(2):
+            kv = torch.empty((2, 1, 8, S, 128), device="cuda")
+            L.loop_cache_read(g, L.LOOP_KIND_FULL, slot, 1, S, kv)
+            k, v = o.kv(slot, 1, S)
+            torch.cuda.synchronize()
+            check(kv[0].cpu().numpy(), k)
+            check(kv[1].cpu().numpy(), v)
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
