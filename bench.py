@@ -1,0 +1,363 @@
+#!/usr/bin/env python
+"""Throughput bench of the looped weight-shared decoder on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole forward path over one batch of synthetic
+input: for a prefill workload, loop_prefill of B sequences x S tokens (56
+layer executions, mHC, attention, linear attention, output head); for the
+decode workload, one loop_decode_step of 64 sequences.  Prints one JSON line
+(rank 0).  With N > 1 (torchrun) every rank runs an independent replica on its
+own GPU (the path shards by sequence; there is no data-path collective) and
+the timing is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import seeded  # noqa: E402
+from seeded import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "loop9b_prefill_b4_s8192"
+DATA = "synthetic: seeded SplitMix64 token ids, random-init N(0, 0.02) bf16 weights of the 9B shape"
+
+
+def args_():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=3)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample-tokens", type=int, default=12)
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def workload_info(name):
+    w = W.WORKLOADS[name]
+    m = dict(w["model"])
+    decode = "decode_steps" in w
+    return w, m, decode
+
+
+def metric_for(name, decode):
+    if decode:
+        return "looped-decoder decode tokens/s at 9B shape", "tokens/s"
+    if W.WORKLOADS[name]["model"]["io_mode"] == 1:
+        return "looped 4-layer group prefill tokens/s at 9B width", "tokens/s"
+    return "looped-decoder prefill tokens/s at 9B shape", "tokens/s"
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- our arm
+
+def run_ours(a, rank, world, local_rank):
+    import torch
+    import looped_weight_shared_b200 as L
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w, m, decode = workload_info(a.workload)
+    B, S, seed = w["batch"], w["seq"], w["seed"]
+    if decode:
+        m.update(max_batch=B, max_ctx=S + a.warmup + 2 * a.steps + 2)
+    else:
+        m.update(max_batch=B, max_ctx=S)
+    cfg = L.make_config(**m)
+    t0 = time.time()
+    g = L.loop_model_create(cfg, seed=seed)
+    create_s = time.time() - t0
+    stream = torch.cuda.current_stream(dev)
+    V, H = m["vocab"], m["hidden"]
+
+    if decode:
+        tok = torch.from_numpy(seeded.tokens(seed, B, S, V)).to(dev)
+        L.loop_prefill(g, tokens=tok, out=torch.empty((B, V), device=dev))
+        nxt = seeded.tokens(seed, B, a.warmup + 2 * a.steps + 2, V, stream=seeded.S_DECODE_TOKENS)
+        step_tok = [torch.from_numpy(nxt[:, i].copy()).to(dev) for i in range(nxt.shape[1])]
+        out = torch.empty((B, V), device=dev)
+        it = iter(step_tok)
+
+        def step():
+            L.loop_decode_step(g, next(it), out)
+        units = B
+    elif m["io_mode"] == 1:
+        hid = torch.from_numpy(seeded.hidden(seed, B, S, H)).to(dev)
+        out = torch.empty((B, S, H), device=dev)
+
+        def step():
+            L.loop_prefill(g, hidden=hid, out=out)
+        units = B * S
+    else:
+        tok = torch.from_numpy(seeded.tokens(seed, B, S, V)).to(dev)
+        out = torch.empty((B, V), device=dev)
+
+        def step():
+            L.loop_prefill(g, tokens=tok, out=out)
+        units = B * S
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    L.loop_timing_read(g, 0, reset=True)
+    L.loop_set_timing(g, True)
+    launches0 = L.loop_launch_count(g)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        for _ in range(a.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    L.loop_set_timing(g, False)
+    launches = L.loop_launch_count(g) - launches0
+    ms = ev0.elapsed_time(ev1) / a.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+        torch.distributed.barrier()
+    value = units * world / (ms / 1e3)
+    classes = {}
+    for ci, cname in enumerate(L.KERNEL_CLASSES):
+        tms, n, work = L.loop_timing_read(g, ci)
+        classes[cname] = {"ms_per_step": tms / a.steps, "launches": n, "work": work}
+    status = L.loop_device_status()
+
+    # e2e: the same step through the C ABI with host buffers (pinned), the
+    # step's inputs copied in and its result read back inside the timed region
+    if decode:
+        host_in = torch.from_numpy(nxt[:, -a.steps:].T.copy()).pin_memory()
+        e2e_out = torch.empty((B, V), pin_memory=True)
+        d_tok = torch.empty((B,), dtype=torch.int32, device=dev)
+        h2d = B * 4
+        d2h = B * V * 4
+    elif m["io_mode"] == 1:
+        host_in = torch.from_numpy(seeded.hidden(seed, B, S, H)).pin_memory()
+        e2e_out = torch.empty((B, S, H), pin_memory=True)
+        d_hid = torch.empty((B, S, H), device=dev)
+        h2d = B * S * H * 4
+        d2h = B * S * H * 4
+    else:
+        host_in = torch.from_numpy(seeded.tokens(seed, B, S, V)).pin_memory()
+        e2e_out = torch.empty((B, V), pin_memory=True)
+        d_tok = torch.empty((B, S), dtype=torch.int32, device=dev)
+        h2d = B * S * 4
+        d2h = B * V * 4
+
+    def e2e_step(i):
+        if decode:
+            d_tok.copy_(host_in[i % host_in.shape[0]], non_blocking=True)
+            L.loop_decode_step(g, d_tok, out)
+        elif m["io_mode"] == 1:
+            d_hid.copy_(host_in, non_blocking=True)
+            L.loop_prefill(g, hidden=d_hid, out=out)
+        else:
+            d_tok.copy_(host_in, non_blocking=True)
+            L.loop_prefill(g, tokens=d_tok, out=out)
+        e2e_out.copy_(out, non_blocking=True)
+
+    e2e_steps = a.steps
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ev0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    L.loop_model_destroy(g)
+    return dict(ms=ms, value=value, classes=classes, clocks=clk.summary(), launches=launches, status=status,
+                e2e_ms=e2e_ms, e2e_value=units * world / (e2e_ms / 1e3), h2d=h2d, d2h=d2h, create_s=create_s,
+                units=units)
+
+
+# ---------------------------------------------------------------------------- oracle (CPU)
+
+def oracle_sample(a, steps=1):
+    """Time the oracle on a bounded sample of the workload on this host's cores."""
+    import numpy as np
+    import oracle
+
+    w, m, decode = workload_info(a.workload)
+    seed = w["seed"]
+    s_tok = a.cpu_sample_tokens
+    mm = dict(m, max_batch=1, max_ctx=s_tok + steps + 1)
+    t0 = time.time()
+    o = oracle.Model(oracle.make_config(**mm), seed=seed)
+    setup = time.time() - t0
+    times = []
+    if decode:
+        tok = seeded.tokens(seed, 1, s_tok, m["vocab"])
+        o.prefill(tok)
+        for i in range(steps):
+            t = time.time()
+            o.decode_step(np.array([int(tok[0, i % s_tok])], dtype=np.int32))
+            times.append(time.time() - t)
+        units = 1
+        sample = (f"decode steps of 1 sequence after a {s_tok}-token prefill at the 9B shape (the workload decodes "
+                  f"64 sequences after 32,768 tokens; the oracle's per-token cost there is higher)")
+    elif m["io_mode"] == 1:
+        h = seeded.hidden(seed, 1, s_tok, m["hidden"])
+        for _ in range(steps):
+            t = time.time()
+            o.prefill(hidden=h)
+            times.append(time.time() - t)
+        units = s_tok
+        sample = f"prefill of 1 x {s_tok} tokens of the workload's model (the workload is {w['batch']} x {w['seq']})"
+    else:
+        tok = seeded.tokens(seed, 1, s_tok, m["vocab"])
+        for _ in range(steps):
+            t = time.time()
+            o.prefill(tok)
+            times.append(time.time() - t)
+        units = s_tok
+        sample = f"prefill of 1 x {s_tok} tokens of the workload's model (the workload is {w['batch']} x {w['seq']})"
+    o.close()
+    return dict(value=units / statistics.mean(times), times=times, sample=sample, setup_s=setup,
+                cores=int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)))
+
+
+# ---------------------------------------------------------------------------- main
+
+def main():
+    a = args_()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w, m, decode = workload_info(a.workload)
+    metric, unit = metric_for(a.workload, decode)
+    config = {"workload": a.workload, "batch": w["batch"], "seq_len": w["seq"],
+              "l2": "inputs larger than L2: 15.6 GB of weights and >1 GB of activations stream through every step",
+              "parallelism": f"replicas x{world}"}
+    if decode:
+        config["decode_context"] = w["seq"]
+
+    if a.impl == "reference":
+        if rank != 0:
+            return
+        r = oracle_sample(a, steps=a.steps)
+        line = {"impl": "reference", "metric": metric, "value": r["value"], "unit": unit, "n_gpus": a.gpus,
+                "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * statistics.mean(r["times"]),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": DATA, "config": config,
+                "cpu_baseline": {"value": r["value"], "unit": unit, "cores": r["cores"], "kind": "oracle",
+                                 "sample": r["sample"]},
+                "e2e": {"value": r["value"], "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    r = run_ours(a, rank, world, local_rank)
+    pk, pk_kind = peaks()
+    g = r["classes"]["gemm"]
+    ach = g["work"] / (g["ms_per_step"] * a.steps) / 1e9 if g["ms_per_step"] > 0 else 0.0
+    peak = pk["bf16_tflops_sustained"]
+    roof = {"bound": "tensor", "kernel": "tcgen05 projection GEMM (all launches in the timed steps)",
+            "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak if peak else None,
+            "peak_kind": f"{pk_kind} sustained bf16", "traffic": None}
+    line = {"metric": metric, "value": r["value"], "unit": unit, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": DATA, "config": config, "clocks": r["clocks"],
+            "roofline": roof,
+            "e2e": {"value": r["e2e_value"], "unit": unit, "h2d_bytes_per_step": r["h2d"],
+                    "d2h_bytes_per_step": r["d2h"]},
+            "gpu_launches": r["launches"],
+            "kernel_ms_per_step": {k: round(v["ms_per_step"], 3) for k, v in r["classes"].items()},
+            "device_status": r["status"]}
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        c = oracle_sample(a, steps=1)
+        line["cpu_baseline"] = {"value": c["value"], "unit": unit, "cores": c["cores"], "kind": "oracle",
+                                "sample": c["sample"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

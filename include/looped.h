@@ -164,6 +164,31 @@ LOOP_API int32_t loop_weight_read(loop_model* m, int32_t index, float* d_out, vo
 LOOP_API int32_t loop_gemm_bf16(const void* d_A, const void* d_W, int64_t M, int64_t N, int64_t K, float* d_C,
                                 int64_t ldc, int32_t use_tensor_cores, void* stream);
 
+/* Kernel classes for loop_timing_read. */
+enum {
+  LOOP_K_GEMM = 0,             /* projection GEMMs and the output head */
+  LOOP_K_ATTENTION = 1,        /* causal GQA attention (prefill and decode) */
+  LOOP_K_LINEAR_ATTENTION = 2, /* gated linear attention */
+  LOOP_K_MHC = 3,              /* mHC prologue */
+  LOOP_K_NORM = 4,             /* RMSNorm, embedding, stream expand/collapse */
+  LOOP_K_OTHER = 5,
+  LOOP_K_CLASSES = 6
+};
+
+/* Enable (1) or disable (0) per-launch timing: while enabled every kernel
+ * the model launches is bracketed by CUDA events on its stream. */
+LOOP_API int32_t loop_set_timing(loop_model* m, int32_t enable);
+
+/* Totals for kernel class `cls` since the last reset: device time in ms,
+ * launches, and algorithmic work (FLOPs for LOOP_K_GEMM, LOOP_K_ATTENTION and
+ * LOOP_K_LINEAR_ATTENTION; bytes that must move for the others).  Waits for
+ * the recorded events.  reset != 0 clears the totals afterwards. */
+LOOP_API int32_t loop_timing_read(loop_model* m, int32_t cls, double* total_ms, int64_t* launches, double* work,
+                                  int32_t reset);
+
+/* Number of kernels this model has launched since it was created. */
+LOOP_API int64_t loop_launch_count(const loop_model* m);
+
 /* Sticky device status word: 0, or the bits of waits that timed out in a
  * kernel (the kernel then returned early).  Reading it synchronises the
  * device.  loop_clear_device_status() resets it. */

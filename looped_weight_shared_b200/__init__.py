@@ -19,11 +19,13 @@ LOOP_F32, LOOP_BF16 = 0, 1
 LOOP_TOKENS_TO_LOGITS, LOOP_HIDDEN_TO_HIDDEN = 0, 1
 LOOP_ALL_POSITIONS = 1
 LOOP_KIND_LINEAR, LOOP_KIND_FULL = 0, 1
+LOOP_K_GEMM, LOOP_K_ATTENTION, LOOP_K_LINEAR_ATTENTION, LOOP_K_MHC, LOOP_K_NORM, LOOP_K_OTHER = range(6)
+KERNEL_CLASSES = ("gemm", "attention", "linear_attention", "mhc", "norm", "other")
 
 API = ("loop_num_exec", "loop_schedule", "loop_num_weights", "loop_model_create", "loop_prefill",
        "loop_decode_step", "mhc_sinkhorn", "loop_model_destroy", "loop_seq_len", "loop_cache_read",
        "loop_weight_read", "loop_device_status", "loop_clear_device_status", "loop_last_error",
-       "loop_gemm_bf16")
+       "loop_gemm_bf16", "loop_set_timing", "loop_timing_read", "loop_launch_count")
 
 
 class loop_config(C.Structure):
@@ -74,6 +76,9 @@ def lib():
             "loop_clear_device_status": (None, []),
             "loop_last_error": (C.c_char_p, []),
             "loop_gemm_bf16": (i32, [vp, vp, C.c_int64, C.c_int64, C.c_int64, vp, C.c_int64, i32, vp]),
+            "loop_set_timing": (i32, [vp, i32]),
+            "loop_timing_read": (i32, [vp, i32, P(C.c_double), P(C.c_int64), P(C.c_double), i32]),
+            "loop_launch_count": (C.c_int64, [vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -190,3 +195,19 @@ def loop_gemm_bf16(A, W, C_out, use_tensor_cores: bool = True, stream=None) -> N
     N = int(W.shape[0])
     _check("loop_gemm_bf16", lib().loop_gemm_bf16(_ptr(A), _ptr(W), M, N, K, _ptr(C_out), int(C_out.stride(0)),
                                                   1 if use_tensor_cores else 0, _stream(stream)))
+
+
+def loop_set_timing(model: int, enable: bool) -> None:
+    _check("loop_set_timing", lib().loop_set_timing(C.c_void_p(model), 1 if enable else 0))
+
+
+def loop_timing_read(model: int, cls: int, reset: bool = False):
+    """(total_ms, launches, work) of kernel class cls."""
+    ms, n, w = C.c_double(), C.c_int64(), C.c_double()
+    _check("loop_timing_read", lib().loop_timing_read(C.c_void_p(model), cls, C.byref(ms), C.byref(n), C.byref(w),
+                                                      1 if reset else 0))
+    return ms.value, n.value, w.value
+
+
+def loop_launch_count(model: int) -> int:
+    return lib().loop_launch_count(C.c_void_p(model))

@@ -144,11 +144,13 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, const EpiP& p) {
       ld_chunk(tacc + 32 * c, v);
       if (!valid) continue;
       float4* h = reinterpret_cast<float4*>(p.c + (int64_t)row * p.N + n);
+      float4 x[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] = h[j];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        float4 x = h[j];
-        x.x += v[4 * j]; x.y += v[4 * j + 1]; x.z += v[4 * j + 2]; x.w += v[4 * j + 3];
-        h[j] = x;
+        x[j].x += v[4 * j]; x[j].y += v[4 * j + 1]; x[j].z += v[4 * j + 2]; x[j].w += v[4 * j + 3];
+        h[j] = x[j];
       }
     }
   } else if constexpr (MODE == Epi::MHC_WRITE) {
@@ -165,21 +167,30 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, const EpiP& p) {
       if (!valid) continue;
       float4* s0 = reinterpret_cast<float4*>(p.s + (int64_t)row * p.N + n);
       float4* s1 = reinterpret_cast<float4*>(p.s + plane + (int64_t)row * p.N + n);
+      // all loads first: s0 and s1 may alias as far as the compiler knows
+      float4 a[8], b[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __ldcs(s0 + j);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) b[j] = __ldcs(s1 + j);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float4 a = s0[j], b = s1[j];
         float4 x, y;
-        x.x = c1.x * a.x + c1.y * b.x + c0.z * v[4 * j + 0];
-        x.y = c1.x * a.y + c1.y * b.y + c0.z * v[4 * j + 1];
-        x.z = c1.x * a.z + c1.y * b.z + c0.z * v[4 * j + 2];
-        x.w = c1.x * a.w + c1.y * b.w + c0.z * v[4 * j + 3];
-        y.x = c1.z * a.x + c1.w * b.x + c0.w * v[4 * j + 0];
-        y.y = c1.z * a.y + c1.w * b.y + c0.w * v[4 * j + 1];
-        y.z = c1.z * a.z + c1.w * b.z + c0.w * v[4 * j + 2];
-        y.w = c1.z * a.w + c1.w * b.w + c0.w * v[4 * j + 3];
-        s0[j] = x;
-        s1[j] = y;
+        x.x = c1.x * a[j].x + c1.y * b[j].x + c0.z * v[4 * j + 0];
+        x.y = c1.x * a[j].y + c1.y * b[j].y + c0.z * v[4 * j + 1];
+        x.z = c1.x * a[j].z + c1.y * b[j].z + c0.z * v[4 * j + 2];
+        x.w = c1.x * a[j].w + c1.y * b[j].w + c0.z * v[4 * j + 3];
+        y.x = c1.z * a[j].x + c1.w * b[j].x + c0.w * v[4 * j + 0];
+        y.y = c1.z * a[j].y + c1.w * b[j].y + c0.w * v[4 * j + 1];
+        y.z = c1.z * a[j].z + c1.w * b[j].z + c0.w * v[4 * j + 2];
+        y.w = c1.z * a[j].w + c1.w * b[j].w + c0.w * v[4 * j + 3];
+        a[j] = x;
+        b[j] = y;
       }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s0[j] = a[j];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s1[j] = b[j];
     }
   } else if constexpr (MODE == Epi::SWIGLU) {
     const int F = p.N / 2;

@@ -154,6 +154,13 @@ void release(Model& m) {
   if (!m.allocs.empty()) cudaDeviceSynchronize();
   for (void* p : m.allocs) cudaFree(p);
   m.allocs.clear();
+  for (auto& t : m.pending) {
+    cudaEventDestroy(t.a);
+    cudaEventDestroy(t.b);
+  }
+  m.pending.clear();
+  for (auto e : m.event_pool) cudaEventDestroy(e);
+  m.event_pool.clear();
 }
 
 void* dev_alloc(Model& m, size_t bytes) {
@@ -280,9 +287,11 @@ int32_t create_impl(const loop_config* cfg, const float* const* hw, uint64_t see
   const int64_t Bm = c.max_batch, ctx = c.max_ctx;
   m.kc.assign(m.n_full, nullptr);
   m.vc.assign(m.n_full, nullptr);
-  for (int i = 0; i < m.n_full; ++i) {
+  for (int i = 0; i < m.n_full; ++i) {  // zeroed: positions never written hold finite values
     LOOP_ALLOC(m.kc[i], void*, Bm * nkv * ctx * hd * es);
     LOOP_ALLOC(m.vc[i], void*, Bm * nkv * ctx * hd * es);
+    LOOP_CU(cudaMemset(m.kc[i], 0, Bm * nkv * ctx * hd * es));
+    LOOP_CU(cudaMemset(m.vc[i], 0, Bm * nkv * ctx * hd * es));
   }
   m.st.assign(m.n_lin, nullptr);
   for (int i = 0; i < m.n_lin; ++i) {
@@ -336,16 +345,104 @@ int32_t create_impl(const loop_config* cfg, const float* const* hw, uint64_t see
 #undef LOOP_RC
 }
 
+cudaEvent_t take_event(Model& m) {
+  if (!m.event_pool.empty()) {
+    cudaEvent_t e = m.event_pool.back();
+    m.event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+
+// Run `launch` (which enqueues `kernels` kernels on st) and account for it.
+template <typename F>
+cudaError_t timed(Model& m, int cls, double work, int kernels, cudaStream_t st, F&& launch) {
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (m.timing) {
+    a = take_event(m);
+    b = take_event(m);
+    if (a) cudaEventRecord(a, st);
+  }
+  cudaError_t err = launch();
+  m.launches += kernels;
+  if (m.timing && a && b) {
+    cudaEventRecord(b, st);
+    m.pending.push_back({cls, work, a, b});
+  }
+  return err;
+}
+
+void drain_timing(Model& m) {
+  for (auto& t : m.pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(t.b) == cudaSuccess && cudaEventElapsedTime(&ms, t.a, t.b) == cudaSuccess) {
+      m.t_ms[t.cls] += ms;
+      m.t_work[t.cls] += t.work;
+      m.t_count[t.cls] += 1;
+    } else {
+      cudaGetLastError();
+    }
+    m.event_pool.push_back(t.a);
+    m.event_pool.push_back(t.b);
+  }
+  m.pending.clear();
+}
+
 // A projection: C = A W^T followed by its epilogue.
 cudaError_t project(Model& m, const void* A, const void* W, int64_t M, int64_t N, int64_t K, const EpiArgs& e,
                     cudaStream_t st) {
   if (M == 0) return cudaSuccess;
-  if (m.use_tc && gemm_tc_supported(M, N, K, e)) return launch_gemm_tc(A, W, M, N, K, e, st);
+  const double flops = 2.0 * (double)M * (double)N * (double)K;
+  if (m.use_tc && gemm_tc_supported(M, N, K, e))
+    return timed(m, LOOP_K_GEMM, flops, 1, st, [&] { return launch_gemm_tc(A, W, M, N, K, e, st); });
   float* C = e.mode == Epi::F32 ? e.c : m.w.cbuf;
   const int64_t ldc = e.mode == Epi::F32 ? e.ldc : N;
-  cudaError_t err = launch_gemm_simt(A, W, bf16_model(m), M, N, K, C, ldc, st);
+  cudaError_t err = timed(m, LOOP_K_GEMM, flops, 1, st,
+                          [&] { return launch_gemm_simt(A, W, bf16_model(m), M, N, K, C, ldc, st); });
   if (err != cudaSuccess) return err;
-  return launch_epilogue_unfused(C, ldc, M, N, e, bf16_model(m), st);
+  if (e.mode == Epi::F32) return cudaSuccess;
+  return timed(m, LOOP_K_OTHER, 0.0, 1, st,
+               [&] { return launch_epilogue_unfused(C, ldc, M, N, e, bf16_model(m), st); });
+}
+
+// Causal GQA attention of the current q against this execution's KV slot.
+cudaError_t attention(Model& m, const void* Kc, const void* Vc, int B, int S, const int32_t* d_start, cudaStream_t st) {
+  const loop_config& c = m.c;
+  const bool bf = bf16_model(m);
+  // algorithmic FLOPs: QK^T and PV over the causal keys, assuming the
+  // sequences start at position 0 for a prefill (S > 1) or at S - 1 keys back
+  const double pairs = (double)B * S * (S + 1) / 2.0;
+  const double flops = 4.0 * pairs * c.head_dim * c.n_q;
+  if (bf && S > 1 && flash_supported(c.head_dim, c.n_q, c.n_kv))  // a prefill: every sequence starts at 0
+    return timed(m, LOOP_K_ATTENTION, flops, 1, st, [&] {
+      return launch_flash_prefill(m.w.q, Kc, Vc, m.w.o, B, S, c.n_q, c.n_kv, c.max_ctx, st);
+    });
+  return timed(m, LOOP_K_ATTENTION, flops, 1, st, [&] {
+    return launch_attention_simple(m.w.q, Kc, Vc, m.w.o, bf, B, S, c.n_q, c.n_kv, c.head_dim, c.max_ctx, d_start, st);
+  });
+}
+
+// Gated linear attention of the current q, k, v against this execution's state slot.
+cudaError_t linear_attention(Model& m, float* state, int B, int S, cudaStream_t st) {
+  const loop_config& c = m.c;
+  const bool bf = bf16_model(m);
+  const double d = c.lin_dim;
+  if (bf && S > 1 && gla_chunk_supported(c.lin_dim)) {
+    // chunked form: Q K^T, (.)V, Q S and K^T V per chunk of 64 tokens
+    const double flops = 4.0 * (double)B * S * c.n_lin * d * (64.0 + d);
+    return timed(m, LOOP_K_LINEAR_ATTENTION, flops, 1, st, [&] {
+      return launch_gla_chunked(m.w.q, m.w.k, m.w.v, m.w.gl, state, m.w.o, B, S, c.n_lin, st);
+    });
+  }
+  const double flops = 4.0 * (double)B * S * c.n_lin * d * d;
+  return timed(m, LOOP_K_LINEAR_ATTENTION, flops, 1, st, [&] {
+    return launch_gla_recurrent(m.w.q, m.w.k, m.w.v, m.w.gl, state, m.w.o, bf, B, S, c.n_lin, c.lin_dim, st);
+  });
 }
 
 // One forward pass over sequences [b0, b0 + B) with S new tokens each,
@@ -358,7 +455,9 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
   const int64_t nl = c.n_lin, ld = c.lin_dim, nq = c.n_q, nkv = c.n_kv, hd = c.head_dim;
   const int64_t es = m.esize;
   Work& w = m.w;
-  if (c.io_mode == LOOP_TOKENS_TO_LOGITS) LOOP_CU(launch_embed(tokens, m.embed, bf, T, (int)H, c.vocab, w.h, st));
+  if (c.io_mode == LOOP_TOKENS_TO_LOGITS)
+    LOOP_CU(timed(m, LOOP_K_NORM, (double)T * H * (es + 4), 1, st,
+                  [&] { return launch_embed(tokens, m.embed, bf, T, (int)H, c.vocab, w.h, st); }));
   else LOOP_CU(cudaMemcpyAsync(w.h, hidden, T * H * 4, cudaMemcpyDeviceToDevice, st));
   const int first_block = c.n_prelude, last_block = c.n_prelude + c.n_block * c.n_loops - 1;
   float* s_buf = w.s;  // streams [2][T][H]
@@ -367,15 +466,19 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
     const int phys = row[0], kind = row[2], slot = row[3], region = row[4];
     const LayerW& L = m.L[phys];
     const bool in_block = region == LOOP_REGION_BLOCK;
-    if (e == first_block) LOOP_CU(launch_expand(w.h, s_buf, T * H, st));
+    if (e == first_block)
+      LOOP_CU(timed(m, LOOP_K_NORM, 12.0 * T * H, 1, st, [&] { return launch_expand(w.h, s_buf, T * H, st); }));
     for (int sub = 0; sub < 2; ++sub) {
       const float* gain = sub == 0 ? L.attn_gain : L.ffn_gain;
       if (in_block) {
         const SiteW& site = m.sites[2 * (phys - c.n_prelude) + sub];
-        LOOP_CU(launch_mhc_prologue(s_buf, T, (int)H, site.gamma, site.phi, gain, c.sinkhorn_iters, c.norm_eps,
-                                    w.coef, w.xh, bf, st));
+        LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), 1, st, [&] {
+          return launch_mhc_prologue(s_buf, T, (int)H, site.gamma, site.phi, gain, c.sinkhorn_iters, c.norm_eps,
+                                     w.coef, w.xh, bf, st);
+        }));
       } else {
-        LOOP_CU(launch_rmsnorm(w.h, T, (int)H, 1, 0, gain, c.norm_eps, w.xh, bf, st));
+        LOOP_CU(timed(m, LOOP_K_NORM, (double)T * H * (4 + es), 1, st,
+                      [&] { return launch_rmsnorm(w.h, T, (int)H, 1, 0, gain, c.norm_eps, w.xh, bf, st); }));
       }
       EpiArgs out_epi;
       if (in_block) {
@@ -396,8 +499,7 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
           qe.rope = m.rope; qe.start = d_start; qe.S = S;
           qe.heads_q = (int)nq; qe.heads_kv = (int)nkv; qe.hd = (int)hd; qe.cache_ctx = c.max_ctx;
           LOOP_CU(project(m, w.xh, L.w_in, T, L.n_in, H, qe, st));
-          LOOP_CU(launch_attention_simple(w.q, Kc, Vc, w.o, bf, B, S, (int)nq, (int)nkv, (int)hd, c.max_ctx, d_start,
-                                          st));
+          LOOP_CU(attention(m, Kc, Vc, B, S, d_start, st));
         } else {
           float* state = m.st[slot] + (int64_t)b0 * nl * ld * ld;
           EpiArgs qe;
@@ -405,7 +507,7 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
           qe.q = w.q; qe.k = w.k; qe.v = w.v; qe.gl = w.gl;
           qe.S = S; qe.n_lin = (int)nl; qe.hd = (int)ld; qe.eps = c.norm_eps;
           LOOP_CU(project(m, w.xh, L.w_in, T, L.n_in, H, qe, st));
-          LOOP_CU(launch_gla_recurrent(w.q, w.k, w.v, w.gl, state, w.o, bf, B, S, (int)nl, (int)ld, st));
+          LOOP_CU(linear_attention(m, state, B, S, st));
         }
         LOOP_CU(project(m, w.o, L.w_o, T, H, L.n_o_in, out_epi, st));
       } else {
@@ -416,7 +518,8 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
         LOOP_CU(project(m, w.a, L.w_down, T, H, F, out_epi, st));
       }
     }
-    if (e == last_block) LOOP_CU(launch_collapse(s_buf, w.h, T * H, st));
+    if (e == last_block)
+      LOOP_CU(timed(m, LOOP_K_NORM, 12.0 * T * H, 1, st, [&] { return launch_collapse(s_buf, w.h, T * H, st); }));
   }
   if (c.io_mode == LOOP_HIDDEN_TO_HIDDEN) {
     LOOP_CU(cudaMemcpyAsync(out, w.h, T * H * 4, cudaMemcpyDeviceToDevice, st));
@@ -424,7 +527,9 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
   }
   const bool all = (flags & LOOP_ALL_POSITIONS) && !last_only;
   const int64_t rows = all ? T : B;
-  LOOP_CU(launch_rmsnorm(w.h, rows, (int)H, all ? 1 : S, all ? 0 : S - 1, m.final_gain, c.norm_eps, w.xh, bf, st));
+  LOOP_CU(timed(m, LOOP_K_NORM, (double)rows * H * (4 + es), 1, st, [&] {
+    return launch_rmsnorm(w.h, rows, (int)H, all ? 1 : S, all ? 0 : S - 1, m.final_gain, c.norm_eps, w.xh, bf, st);
+  }));
   EpiArgs le;
   le.mode = Epi::F32;
   le.c = out;
@@ -495,7 +600,7 @@ int32_t loop_prefill(loop_model* mp, const int32_t* d_tokens, const float* d_hid
                                false, st);
     if (rc != LOOP_OK) return rc;
   }
-  LOOP_CU(launch_set_len(m.d_seq_len, B, S, st));
+  LOOP_CU(timed(m, LOOP_K_OTHER, 0.0, 1, st, [&] { return launch_set_len(m.d_seq_len, B, S, st); }));
   for (int b = 0; b < B; ++b) m.seq_len[b] = S;
   return LOOP_OK;
 }
@@ -511,7 +616,7 @@ int32_t loop_decode_step(loop_model* mp, const int32_t* d_tokens, int32_t B, flo
   cudaStream_t st = (cudaStream_t)stream;
   const int32_t rc = forward(m, d_tokens, nullptr, 0, B, 1, m.d_seq_len, d_logits, 0, true, st);
   if (rc != LOOP_OK) return rc;
-  LOOP_CU(launch_advance(m.d_seq_len, B, st));
+  LOOP_CU(timed(m, LOOP_K_OTHER, 0.0, 1, st, [&] { return launch_advance(m.d_seq_len, B, st); }));
   for (int b = 0; b < B; ++b) m.seq_len[b] += 1;
   return LOOP_OK;
 }
@@ -600,6 +705,28 @@ int32_t loop_weight_read(loop_model* mp, int32_t index, float* d_out, void* stre
   LOOP_CU(cudaMemcpyAsync(d_out, i % 2 == 0 ? s.gamma : s.phi, rows * cols * 4, cudaMemcpyDeviceToDevice, st));
   return LOOP_OK;
 }
+
+int32_t loop_set_timing(loop_model* mp, int32_t enable) {
+  if (!mp) return fail(LOOP_EINVAL, "model is NULL");
+  mp->m.timing = enable != 0;
+  return LOOP_OK;
+}
+
+int32_t loop_timing_read(loop_model* mp, int32_t cls, double* total_ms, int64_t* launches, double* work,
+                         int32_t reset) {
+  if (!mp || cls < 0 || cls >= LOOP_K_CLASSES) return fail(LOOP_EINVAL, "bad model or class");
+  Model& m = mp->m;
+  drain_timing(m);
+  if (total_ms) *total_ms = m.t_ms[cls];
+  if (launches) *launches = m.t_count[cls];
+  if (work) *work = m.t_work[cls];
+  if (reset) {
+    for (int i = 0; i < LOOP_K_CLASSES; ++i) m.t_ms[i] = m.t_work[i] = 0, m.t_count[i] = 0;
+  }
+  return LOOP_OK;
+}
+
+int64_t loop_launch_count(const loop_model* mp) { return mp ? mp->m.launches : -1; }
 
 int32_t loop_device_status(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(LOOP_ECUDA, "device error");

@@ -77,8 +77,22 @@ struct Work {
   int64_t gla_scratch_floats = 0;
 };
 
+struct TimedLaunch {
+  int cls;
+  double work;
+  cudaEvent_t a, b;
+};
+
 struct Model {
   loop_config c{};
+  // launch accounting
+  int64_t launches = 0;
+  bool timing = false;
+  std::vector<TimedLaunch> pending;
+  std::vector<cudaEvent_t> event_pool;
+  double t_ms[LOOP_K_CLASSES] = {};
+  double t_work[LOOP_K_CLASSES] = {};
+  int64_t t_count[LOOP_K_CLASSES] = {};
   int n_phys = 0, n_exec = 0, n_full = 0, n_lin = 0;
   std::vector<int32_t> table;
   size_t esize = 4;
@@ -134,6 +148,16 @@ cudaError_t launch_advance(int32_t* seq_len, int B, cudaStream_t st);
 cudaError_t launch_set_len(int32_t* seq_len, int B, int S, cudaStream_t st);
 cudaError_t launch_weight_to_f32(const void* src, bool bf16, int64_t rows, int64_t cols, int64_t src_row0,
                                  float* dst, cudaStream_t st);
+
+// flash attention for prefill (bf16, head_dim 128, all sequences from position 0)
+bool flash_supported(int hd, int nq, int nkv);
+cudaError_t launch_flash_prefill(const void* q, const void* K, const void* V, void* o, int B, int S, int nq, int nkv,
+                                 int64_t ctx, cudaStream_t st);
+
+// chunked gated linear attention for prefill (bf16, d = 128)
+bool gla_chunk_supported(int d);
+cudaError_t launch_gla_chunked(const void* q, const void* k, const void* v, const float* gl, float* state, void* o,
+                               int B, int S, int nh, cudaStream_t st);
 
 // tcgen05 GEMM (bf16): C = A[M][K] W[N][K]^T with a fused epilogue.  Returns
 // cudaErrorNotSupported when the shapes are outside what it handles.

@@ -23,3 +23,12 @@ def cosine(got, ref) -> float:
 TOL_F32 = 1e-4
 TOL_BF16 = 2e-2
 COS_BF16 = 0.999
+
+
+def noise_floor(name: str) -> dict:
+    """The oracle's own bf16 noise floor for a model (tests/golden/noise_floor.json)."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "noise_floor.json")
+    with open(path) as f:
+        return json.load(f)[name]

@@ -74,3 +74,32 @@ def test_group9b_bf16_matches_oracle(S):
         assert L.loop_device_status() == 0
     finally:
         L.loop_model_destroy(g)
+
+
+MID = dict(hidden=512, ffn=512, vocab=2048, n_q=4, n_kv=2, head_dim=128, n_lin=4, lin_dim=128, dtype=1)
+
+
+@pytest.mark.parametrize("B,S", [(2, 700), (1, 64), (3, 129)])
+def test_mid_bf16_all_positions(B, S):
+    """head_dim 128 (the flash-attention and fused-epilogue shapes) with a
+    narrow model so the oracle stays fast: several ragged query blocks."""
+    m = dict(W.model_config("tiny_fp32", **MID), max_batch=B, max_ctx=S)
+    g = L.loop_model_create(L.make_config(**m), seed=5)
+    try:
+        o = oracle.Model(oracle.make_config(**m), seed=5)
+        tok = seeded.tokens(5, B, S, m["vocab"])
+        ref = o.prefill(tok, all_positions=True)
+        out = torch.empty((B, S, m["vocab"]), device="cuda")
+        L.loop_prefill(g, tokens=torch.from_numpy(tok).cuda(), out=out, flags=L.LOOP_ALL_POSITIONS)
+        torch.cuda.synchronize()
+        check(out.cpu().numpy(), ref)
+        for slot in range(4):
+            kv = torch.empty((2, B, 2, S, 128), device="cuda")
+            L.loop_cache_read(g, L.LOOP_KIND_FULL, slot, B, S, kv)
+            k, v = o.kv(slot, B, S)
+            torch.cuda.synchronize()
+            check(kv[0].cpu().numpy(), k)
+            check(kv[1].cpu().numpy(), v)
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
