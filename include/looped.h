@@ -139,6 +139,23 @@ LOOP_API int32_t loop_decode_step(loop_model* m, const int32_t* d_tokens, int32_
  * Parameters?", section "What does two-stream mHC do?").  n in [1, 8]. */
 LOOP_API int32_t mhc_sinkhorn(const float* d_logits, float* d_out, int32_t count, int32_t n, int32_t iters, void* stream);
 
+/* One mHC read site for T tokens with n = 2 streams ("How Does SenseNova-Loop
+ * Get More Depth Without More Parameters?", section "What does two-stream mHC
+ * do?": how a layer reads from the streams and how they are mixed):
+ *   r = sqrt(mean over both streams of s^2 + eps),  l = ((s / r) * gamma) . Phi,
+ *   H_pre = sigmoid(l[0:2]), H_post = 2 sigmoid(l[2:4]),
+ *   H_res = Sinkhorn_iters(exp(l[4:8] as 2 x 2)),
+ *   x = H_pre[0] s_0 + H_pre[1] s_1,  x_hat = x / sqrt(mean(x^2) + eps) * gain.
+ * d_streams fp32 [2][T][H] (stream 0 rows, then stream 1 rows); d_gamma fp32
+ * [2H]; d_phi fp32 [8][2H] (rows pre0, pre1, post0, post1, res00, res01, res10,
+ * res11); d_gain fp32 [H]; outputs d_coef fp32 [T][8] in that row order and
+ * d_xhat [T][H] (xhat_dtype LOOP_F32 or LOOP_BF16).  d_scratch: device buffer
+ * of at least 18 * T floats owned by the caller (partial projections; its
+ * contents on entry do not matter).  H a multiple of 4, at most 6144. */
+LOOP_API int32_t mhc_prologue(const float* d_streams, int64_t T, int32_t H, const float* d_gamma,
+                              const float* d_phi, const float* d_gain, int32_t iters, float eps, float* d_coef,
+                              void* d_xhat, int32_t xhat_dtype, float* d_scratch, void* stream);
+
 /* Release everything the model owns.  Waits for the model's queued work. */
 LOOP_API void loop_model_destroy(loop_model* m);
 

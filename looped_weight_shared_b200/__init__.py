@@ -25,7 +25,7 @@ KERNEL_CLASSES = ("gemm", "attention", "linear_attention", "mhc", "norm", "other
 API = ("loop_num_exec", "loop_schedule", "loop_num_weights", "loop_model_create", "loop_prefill",
        "loop_decode_step", "mhc_sinkhorn", "loop_model_destroy", "loop_seq_len", "loop_cache_read",
        "loop_weight_read", "loop_device_status", "loop_clear_device_status", "loop_last_error",
-       "loop_gemm_bf16", "loop_set_timing", "loop_timing_read", "loop_launch_count")
+       "loop_gemm_bf16", "loop_set_timing", "loop_timing_read", "loop_launch_count", "mhc_prologue")
 
 
 class loop_config(C.Structure):
@@ -79,6 +79,7 @@ def lib():
             "loop_set_timing": (i32, [vp, i32]),
             "loop_timing_read": (i32, [vp, i32, P(C.c_double), P(C.c_int64), P(C.c_double), i32]),
             "loop_launch_count": (C.c_int64, [vp]),
+            "mhc_prologue": (i32, [vp, C.c_int64, i32, vp, vp, vp, i32, C.c_float, vp, vp, i32, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -211,3 +212,13 @@ def loop_timing_read(model: int, cls: int, reset: bool = False):
 
 def loop_launch_count(model: int) -> int:
     return lib().loop_launch_count(C.c_void_p(model))
+
+
+def mhc_prologue(streams, gamma, phi, gain, coef, xhat, scratch, iters: int = 20, eps: float = 1e-6,
+                 stream=None) -> None:
+    """streams fp32 cuda [2, T, H]; coef fp32 [T, 8]; xhat fp32 or bf16 [T, H]; scratch fp32 >= 18 T."""
+    import torch
+    T, H = int(streams.shape[1]), int(streams.shape[2])
+    dt = LOOP_BF16 if xhat.dtype == torch.bfloat16 else LOOP_F32
+    _check("mhc_prologue", lib().mhc_prologue(_ptr(streams), T, H, _ptr(gamma), _ptr(phi), _ptr(gain), iters, eps,
+                                              _ptr(coef), _ptr(xhat), dt, _ptr(scratch), _stream(stream)))

@@ -208,6 +208,126 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Decode attention (one new query per sequence): split the context into
+// chunks of 128 keys.  CTA (chunk, kv head, sequence) bulk-copies the chunk's
+// K and V rows (contiguous in the cache) into shared memory and scores the 4
+// query heads of the group: each warp takes 32 keys, lanes split the 128
+// dims so every K row is read once and coalesced.  It writes the chunk's
+// unnormalised o, its max m (log2 domain) and sum l; a combine kernel merges
+// the chunks.  K/V are read from HBM exactly once per step.
+// ---------------------------------------------------------------------------
+constexpr int DEC_KEYS = 128, DEC_G = 4, DEC_THREADS = 128;
+constexpr int DEC_SMEM = 2 * DEC_KEYS * D * 2 + DEC_G * D * 4 + DEC_G * DEC_KEYS * 4 + 64 + 128;
+
+__global__ void __launch_bounds__(DEC_THREADS)
+    attn_decode_partial_kernel(const bf16* __restrict__ q, const bf16* __restrict__ K, const bf16* __restrict__ V,
+                               const int32_t* __restrict__ start, int nq, int nkv, int64_t ctx, int nchunks,
+                               float scale_log2, float* __restrict__ po, float* __restrict__ pml, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  bf16* ks = reinterpret_cast<bf16*>(smem);
+  bf16* vs = ks + DEC_KEYS * D;
+  float* qs = reinterpret_cast<float*>(vs + DEC_KEYS * D);  // [G][128]
+  float* ps = qs + DEC_G * D;                                // [G][keys]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(ps + DEC_G * DEC_KEYS);
+  const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = nq / nkv;
+  const int L = start[b] + 1;  // keys 0 .. start[b] (the new token's K/V are already in the cache)
+  const int k0 = chunk * DEC_KEYS;
+  const int64_t out_base = ((int64_t)b * nq + kvh * G) * nchunks + chunk;
+  if (k0 >= L) {  // past this sequence's end: an empty partial
+    if (tid < G) {
+      pml[(out_base + (int64_t)tid * nchunks) * 2] = -INFINITY;
+      pml[(out_base + (int64_t)tid * nchunks) * 2 + 1] = 0.f;
+    }
+    return;
+  }
+  const int nk = min(DEC_KEYS, L - k0);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const int64_t row = ((int64_t)b * nkv + kvh) * ctx + k0;
+    mbar_expect_tx(bar, 2u * nk * D * 2);
+    bulk_load(ks, K + row * D, nk * D * 2, bar);
+    bulk_load(vs, V + row * D, nk * D * 2, bar);
+  }
+  for (int i = tid; i < G * D; i += DEC_THREADS)
+    qs[i] = __bfloat162float(q[((int64_t)b * nq + kvh * G + i / D) * D + i % D]) * scale_log2;
+  const bool ok = mbar_wait(bar, 0, status, STATUS_WAIT_OTHER);
+  if (__syncthreads_or(!ok)) return;
+  // scores: warp w handles keys w, w + 4, ...; lane owns dims 4 lane .. 4 lane + 3
+  float qv[DEC_G][4];
+#pragma unroll
+  for (int h = 0; h < DEC_G; ++h)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) qv[h][e] = qs[h * D + 4 * lane + e];
+  for (int j = warp; j < nk; j += DEC_THREADS / 32) {
+    const uint2 kr = *reinterpret_cast<const uint2*>(ks + j * D + 4 * lane);
+    const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kr.x));
+    const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kr.y));
+#pragma unroll
+    for (int h = 0; h < DEC_G; ++h) {
+      float d = qv[h][0] * k01.x + qv[h][1] * k01.y + qv[h][2] * k23.x + qv[h][3] * k23.y;
+      d = warp_sum(d);
+      if (lane == 0) ps[h * DEC_KEYS + j] = d;
+    }
+  }
+  __syncthreads();
+  // per head: max and exp2 over the chunk (warp h handles head h)
+  if (warp < DEC_G) {
+    const int h = warp;
+    float m = -INFINITY;
+    for (int j = lane; j < nk; j += 32) m = fmaxf(m, ps[h * DEC_KEYS + j]);
+    m = warp_max(m);
+    float l = 0.f;
+    for (int j = lane; j < nk; j += 32) {
+      const float p = ex2(ps[h * DEC_KEYS + j] - m);
+      ps[h * DEC_KEYS + j] = p;
+      l += p;
+    }
+    l = warp_sum(l);
+    if (lane == 0) {
+      pml[(out_base + (int64_t)h * nchunks) * 2] = m;
+      pml[(out_base + (int64_t)h * nchunks) * 2 + 1] = l;
+    }
+  }
+  __syncthreads();
+  // o[h][d] = sum_j p[h][j] V[j][d]: thread t owns dim t
+  float acc[DEC_G] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int j = 0; j < nk; ++j) {
+    const float v = __bfloat162float(vs[j * D + tid]);
+#pragma unroll
+    for (int h = 0; h < DEC_G; ++h) acc[h] += ps[h * DEC_KEYS + j] * v;
+  }
+#pragma unroll
+  for (int h = 0; h < DEC_G; ++h) po[(out_base + (int64_t)h * nchunks) * D + tid] = acc[h];
+}
+
+__global__ void __launch_bounds__(D)
+    attn_decode_combine_kernel(const float* __restrict__ po, const float* __restrict__ pml, int nq, int nchunks,
+                               bf16* __restrict__ out) {
+  const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  const int64_t base = ((int64_t)b * nq + h) * nchunks;
+  float M = -INFINITY;
+  for (int c = 0; c < nchunks; ++c) M = fmaxf(M, pml[(base + c) * 2]);
+  float l = 0.f, o = 0.f;
+  for (int c = 0; c < nchunks; ++c) {
+    const float m = pml[(base + c) * 2];
+    if (m == -INFINITY) continue;
+    const float w = ex2(m - M);
+    l += w * pml[(base + c) * 2 + 1];
+    o += w * po[(base + c) * D + t];
+  }
+  out[((int64_t)b * nq + h) * D + t] = __float2bfloat16_rn(l > 0.f ? o / l : 0.f);
+}
+
 }  // namespace
 
 static PFN_cuTensorMapEncodeTiled_v12000 encoder() {
@@ -257,6 +377,38 @@ cudaError_t launch_flash_prefill(const void* q, const void* K, const void* V, vo
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   dim3 grid((unsigned)((S + BQ - 1) / BQ), (unsigned)nq, (unsigned)B);
   flash_fwd_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, (bf16*)o, S, nq, nkv, ctx, scale_log2, status_ptr());
+  return cudaGetLastError();
+}
+
+bool decode_attention_supported(int hd, int nq, int nkv) { return hd == D && nq == DEC_G * nkv; }
+
+int64_t decode_attention_scratch_floats(int B, int nq, int64_t ctx) {
+  const int64_t nch = (ctx + DEC_KEYS - 1) / DEC_KEYS;
+  return (int64_t)B * nq * nch * (D + 2);
+}
+
+// q [B][nq][1][128]; K/V cache [B][nkv][ctx][128] with the new position
+// already written; start[b] = position of the new token; o [B][nq*128].
+// scratch: decode_attention_scratch_floats(B, nq, ctx) floats.
+cudaError_t launch_attention_decode(const void* q, const void* K, const void* V, void* o, int B, int nq, int nkv,
+                                    int64_t ctx, int max_len, const int32_t* start, float* scratch, cudaStream_t st) {
+  if (B == 0) return cudaSuccess;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(attn_decode_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int nch = (max_len + DEC_KEYS - 1) / DEC_KEYS;
+  float* po = scratch;
+  float* pml = scratch + (int64_t)B * nq * nch * D;
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  dim3 g1((unsigned)nch, (unsigned)nkv, (unsigned)B);
+  attn_decode_partial_kernel<<<g1, DEC_THREADS, DEC_SMEM, st>>>((const bf16*)q, (const bf16*)K, (const bf16*)V, start,
+                                                                nq, nkv, ctx, nch, scale_log2, po, pml, status_ptr());
+  dim3 g2((unsigned)nq, (unsigned)B);
+  attn_decode_combine_kernel<<<g2, D, 0, st>>>(po, pml, nq, nch, (bf16*)o);
   return cudaGetLastError();
 }
 

@@ -365,6 +365,102 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Skinny GEMM for decode (M <= 64 tokens): the weight is the streamed operand.
+// Swap-AB so the weight rows fill the M = 128 side of tcgen05.mma and the
+// tokens are N = 64; each CTA owns one 128-row weight tile and one slice of K
+// (split-K), so even N = 4096 keeps every SM streaming weights.  Output:
+// fp32 partial sums P[split][token][n] (row stride ldp), reduced by the
+// epilogue kernels.
+// ---------------------------------------------------------------------------
+constexpr int SK_BN = 64, SK_STAGES = 6;
+constexpr int SK_A_BYTES = BM * BK * 2;     // weight tile 128 x 64
+constexpr int SK_B_BYTES = SK_BN * BK * 2;  // token tile 64 x 64
+constexpr int SK_STAGE = SK_A_BYTES + SK_B_BYTES;
+constexpr int SK_SMEM = SK_STAGES * SK_STAGE + 1024 + 256;
+constexpr uint32_t SK_IDESC = idesc_bf16_f32(BM, SK_BN);
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmx, int M, int N,
+                       int K, int splits, float* __restrict__ P, int64_t ldp, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sw_ = smem;
+  uint8_t* sx = smem + SK_STAGES * SK_A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SK_STAGES * SK_STAGE);
+  uint64_t* empty = full + SK_STAGES;
+  uint64_t* tfull = empty + SK_STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, split = blockIdx.y;
+  const int kbs = K / BK;
+  const int kb0 = (int)((int64_t)kbs * split / splits), kb1 = (int)((int64_t)kbs * (split + 1) / splits);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SK_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    fence_mbar_init();
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, SK_BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmw);
+    prefetch_tmap(&tmx);
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&empty[stage], phase ^ 1, status, STATUS_WAIT_PRODUCER)) break;
+      mbar_expect_tx(&full[stage], SK_STAGE);
+      tma_load_2d(sw_ + stage * SK_A_BYTES, &tmw, &full[stage], kb * BK, tile * BM);
+      tma_load_2d(sx + stage * SK_B_BYTES, &tmx, &full[stage], kb * BK, 0);
+      if (++stage == SK_STAGES) { stage = 0; phase ^= 1; }
+    }
+  } else if (warp == 1 && lane == 0) {
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&full[stage], phase, status, STATUS_WAIT_MMA)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(sw_ + stage * SK_A_BYTES), b0 = smem_u32(sx + stage * SK_B_BYTES);
+#pragma unroll
+      for (int k = 0; k < BK / 16; ++k)
+        tc_mma_f16(tmem, smem_desc_sw128(a0 + 32 * k, 1024), smem_desc_sw128(b0 + 32 * k, 1024), SK_IDESC,
+                   (kb > kb0 || k > 0) ? 1u : 0u);
+      tc_commit(&empty[stage]);
+      if (++stage == SK_STAGES) { stage = 0; phase ^= 1; }
+    }
+    if (ok && kb1 > kb0) tc_commit(tfull);
+  } else if (warp >= 4) {
+    const int q = warp & 3;
+    const bool got = kb1 > kb0 && mbar_wait(tfull, 0, status, STATUS_WAIT_EPILOGUE);
+    if (__all_sync(0xffffffffu, got)) {
+      tc_fence_after();
+      const int n = tile * BM + 32 * q + lane;
+      float* dst = P + (int64_t)split * M * ldp + n;
+#pragma unroll 1
+      for (int c = 0; c < SK_BN / 32; ++c) {
+        float v[32];
+        ld_chunk(tmem + ((uint32_t)(32 * q) << 16) + 32 * c, v);
+        if (n < N) {
+          for (int j = 0; j < 32 && 32 * c + j < M; ++j) dst[(int64_t)(32 * c + j) * ldp] = v[j];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, SK_BN);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -422,6 +518,30 @@ cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, int M, int
 }
 
 }  // namespace
+
+bool gemm_skinny_supported(int64_t M, int64_t N, int64_t K) { return M >= 1 && M <= SK_BN && K % BK == 0 && N > 0; }
+
+int gemm_skinny_splits(int64_t N, int64_t K) {
+  const int64_t tiles = (N + BM - 1) / BM, kbs = K / BK;
+  int64_t s = (2 * (int64_t)num_sms() + tiles - 1) / tiles;
+  return (int)std::max<int64_t>(1, std::min<int64_t>({s, kbs, 32}));
+}
+
+cudaError_t launch_gemm_skinny(const void* X, const void* W, int64_t M, int64_t N, int64_t K, int splits, float* P,
+                               int64_t ldp, cudaStream_t st) {
+  if (!gemm_skinny_supported(M, N, K) || splits < 1) return cudaErrorNotSupported;
+  CUtensorMap mw, mx;
+  if (!make_map(&mw, W, N, K, BM) || !make_map(&mx, X, M, K, SK_BN)) return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_skinny_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SK_SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((unsigned)((N + BM - 1) / BM), (unsigned)splits);
+  gemm_skinny_kernel<<<grid, THREADS, SK_SMEM, st>>>(mw, mx, (int)M, (int)N, (int)K, splits, P, ldp, status_ptr());
+  return cudaGetLastError();
+}
 
 bool gemm_tc_supported(int64_t M, int64_t N, int64_t K, const EpiArgs& e) {
   if (M <= 0 || K % BK != 0 || M > (int64_t)1 << 30 || N > (int64_t)1 << 30) return false;

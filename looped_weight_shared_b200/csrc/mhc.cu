@@ -217,129 +217,145 @@ cudaError_t launch_sinkhorn(const float* l, float* out, int64_t count, int n, in
 }
 
 // ---------------------------------------------------------------------------
-// Fused mHC prologue for n = 2 streams.  One CTA handles TOK tokens so the
-// projection Phi [8][2H] is read once per TOK tokens.  Pass 1 accumulates the
-// squared norm and the 8 projections of (s * gamma); one thread per token
-// then forms the coefficients (Sinkhorn included); pass 2 reads
-// x = H_pre[0] s_0 + H_pre[1] s_1 and writes RMSNorm(x) * gain.
+// mHC prologue for n = 2 streams, in two HBM-streaming kernels.
+//
+// (A) mhc_partial: the flattened stream vector u = (s_0, s_1) of a token has
+//     2H entries; CTA (blk, half) keeps half of Phi and gamma (H entries each,
+//     fp32, 8 x H + H floats) in shared memory and every warp streams 8 tokens
+//     of that half with float4 loads, so each Phi value read is used 8 times.
+//     It writes, per token and half, the 8 partial projections
+//     sum_i s_i gamma_i Phi_ci and the partial sum of squares.
+// (B) mhc_read: one warp per token folds the two halves into
+//     l = (sum / r), r = sqrt(sum of squares / 2H + eps), forms H_pre, H_post
+//     and H_res = Sinkhorn(exp(l[4:8])), then reads x = H_pre0 s_0 + H_pre1 s_1
+//     and writes RMSNorm(x) * gain.  The stream rows are read twice (sum of
+//     squares, then the write), the second time from L1/L2.
 // ---------------------------------------------------------------------------
-constexpr int MHC_TOK = 8;
-constexpr int MHC_THREADS = 256;
+constexpr int MHCA_WARPS = 8, MHCA_TOK = 8;  // tokens per warp
+constexpr int MHCA_THREADS = MHCA_WARPS * 32;
+constexpr int MHCB_WARPS = 8;
 
-template <typename T>
-__global__ void __launch_bounds__(MHC_THREADS) mhc_prologue_kernel(const float* __restrict__ s, int64_t Ttot, int H,
-                                                                   const float* __restrict__ gamma,
-                                                                   const float* __restrict__ phi,
-                                                                   const float* __restrict__ gain, int iters,
-                                                                   float eps, float* __restrict__ coef,
-                                                                   T* __restrict__ xh) {
-  __shared__ float red[MHC_THREADS / 32][MHC_TOK][9];
-  __shared__ float cf[MHC_TOK][8];
-  __shared__ float nrm[MHC_TOK];
-  const int64_t t0 = (int64_t)blockIdx.x * MHC_TOK;
-  const int ntok = (int)(Ttot - t0 < MHC_TOK ? Ttot - t0 : MHC_TOK);
-  const int D = 2 * H;
-  float acc[MHC_TOK][9];
+__global__ void __launch_bounds__(MHCA_THREADS, 1)
+    mhc_partial_kernel(const float* __restrict__ s, int64_t T, int H, const float* __restrict__ gamma,
+                       const float* __restrict__ phi, float* __restrict__ part) {
+  extern __shared__ float4 sm4[];
+  const int half = blockIdx.y;
+  const int H4 = H / 4, D = 2 * H;
+  float4* sphi = sm4;            // [8][H4]
+  float4* sgam = sm4 + 8 * H4;   // [H4]
+  for (int i = threadIdx.x; i < H4; i += MHCA_THREADS) {
 #pragma unroll
-  for (int j = 0; j < MHC_TOK; ++j)
+    for (int c = 0; c < 8; ++c)
+      sphi[c * H4 + i] = reinterpret_cast<const float4*>(phi + (int64_t)c * D + (int64_t)half * H)[i];
+    sgam[i] = reinterpret_cast<const float4*>(gamma + (int64_t)half * H)[i];
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t0 = ((int64_t)blockIdx.x * MHCA_WARPS + warp) * MHCA_TOK;
+  if (t0 >= T) return;
+  const int ntok = (int)(T - t0 < MHCA_TOK ? T - t0 : MHCA_TOK);
+  const float4* base = reinterpret_cast<const float4*>(s + ((int64_t)half * T + t0) * H);
+  float acc[MHCA_TOK][9];
+#pragma unroll
+  for (int j = 0; j < MHCA_TOK; ++j)
 #pragma unroll
     for (int c = 0; c < 9; ++c) acc[j][c] = 0.f;
-
-  for (int i = threadIdx.x; i < D; i += MHC_THREADS) {
-    const int stream = i >= H ? 1 : 0;
-    const int col = i - stream * H;
-    float ph[8];
+#pragma unroll 2
+  for (int f = lane; f < H4; f += 32) {
+    float4 v[MHCA_TOK];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) ph[c] = phi[(int64_t)c * D + i];
-    const float g = gamma[i];
+    for (int j = 0; j < MHCA_TOK; ++j) v[j] = j < ntok ? __ldcs(base + (int64_t)j * H4 + f) : make_float4(0, 0, 0, 0);
+    const float4 g = sgam[f];
 #pragma unroll
-    for (int j = 0; j < MHC_TOK; ++j) {
-      if (j < ntok) {
-        const float v = s[((int64_t)stream * Ttot + t0 + j) * H + col];
-        acc[j][8] += v * v;
-        const float w = v * g;
+    for (int c = 0; c < 8; ++c) {
+      const float4 p = sphi[c * H4 + f];
+      const float4 w = make_float4(p.x * g.x, p.y * g.y, p.z * g.z, p.w * g.w);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[j][c] += w * ph[c];
-      }
+      for (int j = 0; j < MHCA_TOK; ++j) acc[j][c] += v[j].x * w.x + v[j].y * w.y + v[j].z * w.z + v[j].w * w.w;
     }
-  }
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 #pragma unroll
-  for (int j = 0; j < MHC_TOK; ++j)
+    for (int j = 0; j < MHCA_TOK; ++j) acc[j][8] += v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
+  }
+#pragma unroll
+  for (int j = 0; j < MHCA_TOK; ++j)
 #pragma unroll
     for (int c = 0; c < 9; ++c) {
       const float r = warp_sum(acc[j][c]);
-      if (lane == 0) red[wid][j][c] = r;
+      if (lane == c && j < ntok) part[((t0 + j) * 2 + half) * 9 + c] = r;
     }
-  __syncthreads();
-  if (threadIdx.x < ntok) {
-    const int j = threadIdx.x;
-    float tot[9];
-    for (int c = 0; c < 9; ++c) {
-      float a = 0.f;
-      for (int w = 0; w < MHC_THREADS / 32; ++w) a += red[w][j][c];
-      tot[c] = a;
-    }
-    const float rinv = rsqrtf(tot[8] / D + eps);
-    float l[8];
-    for (int c = 0; c < 8; ++c) l[c] = tot[c] * rinv;
-    float P[4];
-    sinkhorn_fixed<2>(l + 4, P, iters);
-    cf[j][0] = sigmoidf_(l[0]);
-    cf[j][1] = sigmoidf_(l[1]);
-    cf[j][2] = 2.f * sigmoidf_(l[2]);
-    cf[j][3] = 2.f * sigmoidf_(l[3]);
-    for (int c = 0; c < 4; ++c) cf[j][4 + c] = P[c];
-    for (int c = 0; c < 8; ++c) coef[(t0 + j) * 8 + c] = cf[j][c];
-  }
-  __syncthreads();
-  // pass 2: x = pre0 s0 + pre1 s1, then RMSNorm(x) * gain
-  float ss[MHC_TOK];
+}
+
+template <typename T>
+__global__ void __launch_bounds__(MHCB_WARPS * 32)
+    mhc_read_kernel(const float* __restrict__ s, int64_t Ttot, int H, const float* __restrict__ part,
+                    const float* __restrict__ gain, int iters, float eps, float* __restrict__ coef, T* __restrict__ xh) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * MHCB_WARPS + warp;
+  if (t >= Ttot) return;
+  const float* pp = part + t * 18;
+  float tot[9];
 #pragma unroll
-  for (int j = 0; j < MHC_TOK; ++j) ss[j] = 0.f;
-  for (int i = threadIdx.x; i < H; i += MHC_THREADS) {
+  for (int c = 0; c < 9; ++c) tot[c] = pp[c] + pp[9 + c];
+  const float rinv = rsqrtf(tot[8] / (2 * H) + eps);
+  float l[8];
 #pragma unroll
-    for (int j = 0; j < MHC_TOK; ++j) {
-      if (j < ntok) {
-        const float x = cf[j][0] * s[(t0 + j) * H + i] + cf[j][1] * s[(Ttot + t0 + j) * H + i];
-        ss[j] += x * x;
-      }
-    }
+  for (int c = 0; c < 8; ++c) l[c] = tot[c] * rinv;
+  float P[4];
+  sinkhorn_fixed<2>(l + 4, P, iters);  // every lane computes the same coefficients
+  const float pre0 = sigmoidf_(l[0]), pre1 = sigmoidf_(l[1]);
+  if (lane < 8) {
+    const float v = lane == 0 ? pre0 : lane == 1 ? pre1 : lane == 2 ? 2.f * sigmoidf_(l[2])
+                  : lane == 3 ? 2.f * sigmoidf_(l[3]) : P[lane - 4];
+    coef[t * 8 + lane] = v;
   }
-  __syncthreads();
-#pragma unroll
-  for (int j = 0; j < MHC_TOK; ++j) {
-    const float r = warp_sum(ss[j]);
-    if (lane == 0) red[wid][j][0] = r;
+  const int H4 = H / 4;
+  const float4* s0 = reinterpret_cast<const float4*>(s + t * H);
+  const float4* s1 = reinterpret_cast<const float4*>(s + (Ttot + t) * H);
+  float ss = 0.f;
+#pragma unroll 4
+  for (int f = lane; f < H4; f += 32) {
+    const float4 a = s0[f], b = s1[f];
+    const float x0 = pre0 * a.x + pre1 * b.x, x1 = pre0 * a.y + pre1 * b.y;
+    const float x2 = pre0 * a.z + pre1 * b.z, x3 = pre0 * a.w + pre1 * b.w;
+    ss += x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3;
   }
-  __syncthreads();
-  if (threadIdx.x < ntok) {
-    float a = 0.f;
-    for (int w = 0; w < MHC_THREADS / 32; ++w) a += red[w][threadIdx.x][0];
-    nrm[threadIdx.x] = rsqrtf(a / H + eps);
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < H; i += MHC_THREADS) {
-    const float gi = gain[i];
-#pragma unroll
-    for (int j = 0; j < MHC_TOK; ++j) {
-      if (j < ntok) {
-        const float x = cf[j][0] * s[(t0 + j) * H + i] + cf[j][1] * s[(Ttot + t0 + j) * H + i];
-        xh[(t0 + j) * H + i] = from_f<T>(x * nrm[j] * gi);
-      }
+  ss = warp_sum(ss);
+  const float nrm = rsqrtf(ss / H + eps);
+  const float4* g4 = reinterpret_cast<const float4*>(gain);
+#pragma unroll 4
+  for (int f = lane; f < H4; f += 32) {
+    const float4 a = s0[f], b = s1[f], g = g4[f];
+    const float x0 = (pre0 * a.x + pre1 * b.x) * nrm * g.x, x1 = (pre0 * a.y + pre1 * b.y) * nrm * g.y;
+    const float x2 = (pre0 * a.z + pre1 * b.z) * nrm * g.z, x3 = (pre0 * a.w + pre1 * b.w) * nrm * g.w;
+    if constexpr (sizeof(T) == 2) {
+      uint2 u;
+      u.x = pack_bf16x2(x0, x1);
+      u.y = pack_bf16x2(x2, x3);
+      reinterpret_cast<uint2*>(xh + t * H)[f] = u;
+    } else {
+      reinterpret_cast<float4*>(xh + t * H)[f] = make_float4(x0, x1, x2, x3);
     }
   }
 }
 
+size_t mhc_partial_smem(int H) { return (size_t)9 * H * sizeof(float); }
+
 cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf,
-                                cudaStream_t st) {
+                                float* part, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  const unsigned g = (unsigned)((T + MHC_TOK - 1) / MHC_TOK);
+  if (H % 4 != 0 || mhc_partial_smem(H) > 220 * 1024) return cudaErrorInvalidValue;
+  const int smem = (int)mhc_partial_smem(H);
+  cudaError_t e = cudaFuncSetAttribute(mhc_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t per_cta = (int64_t)MHCA_WARPS * MHCA_TOK;
+  dim3 ga((unsigned)((T + per_cta - 1) / per_cta), 2);
+  mhc_partial_kernel<<<ga, MHCA_THREADS, smem, st>>>(s, T, H, gamma, phi, part);
+  const unsigned gb = (unsigned)((T + MHCB_WARPS - 1) / MHCB_WARPS);
   if (bf)
-    mhc_prologue_kernel<bf16><<<g, MHC_THREADS, 0, st>>>(s, T, H, gamma, phi, gain, iters, eps, coef, (bf16*)xh);
+    mhc_read_kernel<bf16><<<gb, MHCB_WARPS * 32, 0, st>>>(s, T, H, part, gain, iters, eps, coef, (bf16*)xh);
   else
-    mhc_prologue_kernel<float><<<g, MHC_THREADS, 0, st>>>(s, T, H, gamma, phi, gain, iters, eps, coef, (float*)xh);
+    mhc_read_kernel<float><<<gb, MHCB_WARPS * 32, 0, st>>>(s, T, H, part, gain, iters, eps, coef, (float*)xh);
   return cudaGetLastError();
 }
 

@@ -62,6 +62,7 @@ bool valid(const loop_config* c) {
 const char* unsupported(const loop_config* c) {
   if (c->n_streams != 2) return "this build runs n_streams == 2";
   if (c->hidden % 4 != 0) return "hidden must be a multiple of 4";
+  if ((size_t)9 * c->hidden * 4 > 220 * 1024) return "hidden must be <= 6144 (mHC prologue keeps Phi in shared memory)";
   if (c->ffn % 128 != 0) return "ffn must be a multiple of 128";
   if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return "head_dim must be 32, 64 or 128";
   if (c->lin_dim > 256) return "lin_dim must be <= 256";
@@ -312,6 +313,15 @@ int32_t create_impl(const loop_config* cfg, const float* const* hw, uint64_t see
   LOOP_ALLOC(w.s, float*, 2 * T * H * 4);
   LOOP_ALLOC(w.xh, void*, T * H * es);
   LOOP_ALLOC(w.coef, float*, T * 8 * 4);
+  LOOP_ALLOC(w.mhc_part, float*, T * 18 * 4);
+  if (m.use_tc && H % 64 == 0) {  // decode GEMM partials: up to 32 splits x 64 tokens x the widest projection
+    int64_t maxn = std::max<int64_t>(2 * F, H);
+    for (auto& L : m.L) maxn = std::max(maxn, L.n_in);
+    w.cpart_floats = 32 * 64 * maxn;
+    LOOP_ALLOC(w.cpart, float*, w.cpart_floats * 4);
+  }
+  if (bf && decode_attention_supported((int)hd, (int)nq, (int)nkv))
+    LOOP_ALLOC(w.dec_attn, float*, decode_attention_scratch_floats((int)Bm, (int)nq, ctx) * 4);
   LOOP_ALLOC(w.q, void*, T * qw * es);
   LOOP_ALLOC(w.k, void*, T * nl * ld * es);
   LOOP_ALLOC(w.v, void*, T * nl * ld * es);
@@ -398,6 +408,21 @@ cudaError_t project(Model& m, const void* A, const void* W, int64_t M, int64_t N
                     cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const double flops = 2.0 * (double)M * (double)N * (double)K;
+  if (m.decoding && m.use_tc && m.w.cpart && gemm_skinny_supported(M, N, K)) {
+    // decode: weight-streaming split-K GEMM, then the epilogue over the partials
+    // (prefills never take it, so a prefill row is computed the same way
+    // whatever the batch and length)
+    const int splits = gemm_skinny_splits(N, K);
+    const bool direct = e.mode == Epi::F32 && splits == 1;
+    float* P = direct ? e.c : m.w.cpart;
+    const int64_t ldp = direct ? e.ldc : N;
+    if (!direct && (int64_t)splits * M * N > m.w.cpart_floats) return cudaErrorInvalidValue;
+    cudaError_t err = timed(m, LOOP_K_GEMM, flops, 1, st,
+                            [&] { return launch_gemm_skinny(A, W, M, N, K, splits, P, ldp, st); });
+    if (err != cudaSuccess || direct) return err;
+    return timed(m, LOOP_K_OTHER, 0.0, 1, st,
+                 [&] { return launch_epilogue_unfused(P, N, M, N, e, bf16_model(m), st, splits); });
+  }
   if (m.use_tc && gemm_tc_supported(M, N, K, e))
     return timed(m, LOOP_K_GEMM, flops, 1, st, [&] { return launch_gemm_tc(A, W, M, N, K, e, st); });
   float* C = e.mode == Epi::F32 ? e.c : m.w.cbuf;
@@ -418,6 +443,21 @@ cudaError_t attention(Model& m, const void* Kc, const void* Vc, int B, int S, co
   // sequences start at position 0 for a prefill (S > 1) or at S - 1 keys back
   const double pairs = (double)B * S * (S + 1) / 2.0;
   const double flops = 4.0 * pairs * c.head_dim * c.n_q;
+  if (bf && S == 1 && m.w.dec_attn && decode_attention_supported(c.head_dim, c.n_q, c.n_kv)) {
+    // one new token per sequence: its key position is seq_len[b]; the keys
+    // read are the contexts (+1) of the B sequences
+    int max_len = 0;
+    double keys = 0;
+    for (int b = 0; b < B; ++b) {
+      max_len = std::max(max_len, m.seq_len[b] + 1);
+      keys += m.seq_len[b] + 1;
+    }
+    const double dflops = 4.0 * keys * c.head_dim * c.n_q;
+    return timed(m, LOOP_K_ATTENTION, dflops, 2, st, [&] {
+      return launch_attention_decode(m.w.q, Kc, Vc, m.w.o, B, c.n_q, c.n_kv, c.max_ctx, max_len, d_start,
+                                     m.w.dec_attn, st);
+    });
+  }
   if (bf && S > 1 && flash_supported(c.head_dim, c.n_q, c.n_kv))  // a prefill: every sequence starts at 0
     return timed(m, LOOP_K_ATTENTION, flops, 1, st, [&] {
       return launch_flash_prefill(m.w.q, Kc, Vc, m.w.o, B, S, c.n_q, c.n_kv, c.max_ctx, st);
@@ -472,9 +512,9 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
       const float* gain = sub == 0 ? L.attn_gain : L.ffn_gain;
       if (in_block) {
         const SiteW& site = m.sites[2 * (phys - c.n_prelude) + sub];
-        LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), 1, st, [&] {
+        LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), 2, st, [&] {
           return launch_mhc_prologue(s_buf, T, (int)H, site.gamma, site.phi, gain, c.sinkhorn_iters, c.norm_eps,
-                                     w.coef, w.xh, bf, st);
+                                     w.coef, w.xh, bf, w.mhc_part, st);
         }));
       } else {
         LOOP_CU(timed(m, LOOP_K_NORM, (double)T * H * (4 + es), 1, st,
@@ -614,7 +654,9 @@ int32_t loop_decode_step(loop_model* mp, const int32_t* d_tokens, int32_t B, flo
   for (int b = 0; b < B; ++b)
     if (m.seq_len[b] + 1 > m.c.max_ctx) return fail(LOOP_ERANGE, "sequence would pass max_ctx");
   cudaStream_t st = (cudaStream_t)stream;
+  m.decoding = true;
   const int32_t rc = forward(m, d_tokens, nullptr, 0, B, 1, m.d_seq_len, d_logits, 0, true, st);
+  m.decoding = false;
   if (rc != LOOP_OK) return rc;
   LOOP_CU(timed(m, LOOP_K_OTHER, 0.0, 1, st, [&] { return launch_advance(m.d_seq_len, B, st); }));
   for (int b = 0; b < B; ++b) m.seq_len[b] += 1;
@@ -625,6 +667,19 @@ int32_t mhc_sinkhorn(const float* d_logits, float* d_out, int32_t count, int32_t
   if (!d_logits || !d_out) return fail(LOOP_EINVAL, "NULL argument");
   if (count < 0 || n < 1 || n > 8 || iters < 0) return fail(LOOP_EINVAL, "count >= 0, 1 <= n <= 8, iters >= 0");
   LOOP_CU(launch_sinkhorn(d_logits, d_out, count, n, iters, (cudaStream_t)stream));
+  return LOOP_OK;
+}
+
+int32_t mhc_prologue(const float* d_streams, int64_t T, int32_t H, const float* d_gamma, const float* d_phi,
+                     const float* d_gain, int32_t iters, float eps, float* d_coef, void* d_xhat, int32_t xhat_dtype,
+                     float* d_scratch, void* stream) {
+  if (!d_streams || !d_gamma || !d_phi || !d_gain || !d_coef || !d_xhat || !d_scratch)
+    return fail(LOOP_EINVAL, "NULL argument");
+  if (T < 0 || H <= 0 || H % 4 != 0 || mhc_partial_smem(H) > 220 * 1024 || iters < 0 || !(eps >= 0.f))
+    return fail(LOOP_EINVAL, "T >= 0, H a multiple of 4 and <= 6144, iters >= 0, eps >= 0");
+  if (xhat_dtype != LOOP_F32 && xhat_dtype != LOOP_BF16) return fail(LOOP_EINVAL, "bad xhat_dtype");
+  LOOP_CU(launch_mhc_prologue(d_streams, T, H, d_gamma, d_phi, d_gain, iters, eps, d_coef, d_xhat,
+                              xhat_dtype == LOOP_BF16, d_scratch, (cudaStream_t)stream));
   return LOOP_OK;
 }
 

@@ -73,8 +73,10 @@ struct Work {
   float* cbuf = nullptr;    // [T][max N] projection scratch of the unfused path
   void* xf = nullptr;       // [rows][H] final-norm output
   int32_t* zeros = nullptr; // start positions of a prefill (all 0)
-  float* gla_scratch = nullptr;
-  int64_t gla_scratch_floats = 0;
+  float* mhc_part = nullptr;  // [T][2][9] partial projections of the mHC prologue
+  float* cpart = nullptr;     // split-K partial sums of the decode GEMM [32][64][max N]
+  int64_t cpart_floats = 0;
+  float* dec_attn = nullptr;  // decode attention chunk partials [B][n_q][ctx / 128][130]
 };
 
 struct TimedLaunch {
@@ -108,6 +110,7 @@ struct Model {
   Work w;
   std::vector<void*> allocs;
   bool use_tc = false;          // tcgen05 path for bf16 projections
+  bool decoding = false;        // inside loop_decode_step: projections use the decode GEMM
 };
 
 bool bf16_model(const Model& m);
@@ -125,17 +128,20 @@ cudaError_t launch_embed(const int32_t* tok, const void* E, bool bf16, int64_t T
                          cudaStream_t st);
 cudaError_t launch_rmsnorm(const float* x, int64_t rows, int H, int64_t row_step, int64_t row_off,
                            const float* gain, float eps, void* y, bool bf16, cudaStream_t st);
+// two kernels; `part` is scratch of 18 floats per token
 cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf16,
-                                cudaStream_t st);
+                                float* part, cudaStream_t st);
+size_t mhc_partial_smem(int H);
 cudaError_t launch_expand(const float* h, float* s, int64_t n, cudaStream_t st);
 cudaError_t launch_collapse(const float* s, float* h, int64_t n, cudaStream_t st);
 cudaError_t launch_sinkhorn(const float* l, float* out, int64_t count, int n, int iters, cudaStream_t st);
 
 cudaError_t launch_gemm_simt(const void* A, const void* W, bool bf16, int64_t M, int64_t N, int64_t K,
                              float* C, int64_t ldc, cudaStream_t st);
+// C holds `splits` slices of M x ldc (split-K partial sums, added in order).
 cudaError_t launch_epilogue_unfused(const float* C, int64_t ldc, int64_t M, int64_t N, const EpiArgs& e, bool bf16,
-                                    cudaStream_t st);
+                                    cudaStream_t st, int splits = 1);
 cudaError_t launch_attention_simple(const void* q, const void* K, const void* V, void* o, bool bf16, int B, int S,
                                     int nq, int nkv, int hd, int64_t cache_ctx, const int32_t* start,
                                     cudaStream_t st);
@@ -154,6 +160,12 @@ bool flash_supported(int hd, int nq, int nkv);
 cudaError_t launch_flash_prefill(const void* q, const void* K, const void* V, void* o, int B, int S, int nq, int nkv,
                                  int64_t ctx, cudaStream_t st);
 
+// decode attention (flash-decoding over 128-key chunks; bf16, head_dim 128, group 4)
+bool decode_attention_supported(int hd, int nq, int nkv);
+int64_t decode_attention_scratch_floats(int B, int nq, int64_t ctx);
+cudaError_t launch_attention_decode(const void* q, const void* K, const void* V, void* o, int B, int nq, int nkv,
+                                    int64_t ctx, int max_len, const int32_t* start, float* scratch, cudaStream_t st);
+
 // chunked gated linear attention for prefill (bf16, d = 128)
 bool gla_chunk_supported(int d);
 cudaError_t launch_gla_chunked(const void* q, const void* k, const void* v, const float* gl, float* state, void* o,
@@ -164,5 +176,11 @@ cudaError_t launch_gla_chunked(const void* q, const void* k, const void* v, cons
 cudaError_t launch_gemm_tc(const void* A, const void* W, int64_t M, int64_t N, int64_t K, const EpiArgs& e,
                            cudaStream_t st);
 bool gemm_tc_supported(int64_t M, int64_t N, int64_t K, const EpiArgs& e);
+
+// decode GEMM (M <= 64 tokens): swap-AB, split-K; P[split][M][ldp] fp32 partials
+bool gemm_skinny_supported(int64_t M, int64_t N, int64_t K);
+int gemm_skinny_splits(int64_t N, int64_t K);
+cudaError_t launch_gemm_skinny(const void* X, const void* W, int64_t M, int64_t N, int64_t K, int splits, float* P,
+                               int64_t ldp, cudaStream_t st);
 
 }  // namespace loopk

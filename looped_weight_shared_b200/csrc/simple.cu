@@ -64,22 +64,41 @@ cudaError_t launch_gemm_simt(const void* A, const void* W, bool bf, int64_t M, i
 }
 
 // ---------------------------------------------------------------------------
-// epilogues over the scratch C
+// epilogues over the scratch C (optionally `splits` split-K slices of M x ldc
+// each, summed in slice order)
 // ---------------------------------------------------------------------------
-__global__ void epi_resid_kernel(const float* C, int64_t ldc, int64_t M, int64_t N, float* h) {
+struct CView {
+  const float* c;
+  int64_t ldc, slice;
+  int splits;
+  LOOP_DEV float operator()(int64_t r, int64_t col) const {
+    float v = c[r * ldc + col];
+    for (int k = 1; k < splits; ++k) v += c[k * slice + r * ldc + col];
+    return v;
+  }
+};
+__global__ void epi_resid_kernel(CView C, int64_t M, int64_t N, float* h) {
   const int64_t n = M * N;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / N, c = i % N;
-    h[i] += C[r * ldc + c];
+    h[i] += C(r, c);
   }
 }
 
-__global__ void epi_mhc_kernel(const float* C, int64_t ldc, int64_t M, int64_t N, float* s, const float* coef) {
+__global__ void epi_f32_kernel(CView C, int64_t M, int64_t N, float* out, int64_t ldo) {
+  const int64_t n = M * N;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / N, c = i % N;
+    out[r * ldo + c] = C(r, c);
+  }
+}
+
+__global__ void epi_mhc_kernel(CView C, int64_t M, int64_t N, float* s, const float* coef) {
   const int64_t n = M * N;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / N, c = i % N;
     const float* cf = coef + r * 8;
-    const float y = C[r * ldc + c];
+    const float y = C(r, c);
     const float s0 = s[i], s1 = s[n + i];
     s[i] = cf[4] * s0 + cf[5] * s1 + cf[2] * y;
     s[n + i] = cf[6] * s0 + cf[7] * s1 + cf[3] * y;
@@ -87,30 +106,29 @@ __global__ void epi_mhc_kernel(const float* C, int64_t ldc, int64_t M, int64_t N
 }
 
 template <typename T>
-__global__ void epi_swiglu_kernel(const float* C, int64_t ldc, int64_t M, int64_t F, T* a) {
+__global__ void epi_swiglu_kernel(CView C, int64_t M, int64_t F, T* a) {
   const int64_t n = M * F;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / F, f = i % F;
     const int64_t blk = f / 128, j = f % 128;
-    const float g = C[r * ldc + blk * 256 + j], u = C[r * ldc + blk * 256 + 128 + j];
+    const float g = C(r, blk * 256 + j), u = C(r, blk * 256 + 128 + j);
     a[i] = from_f<T>(g * sigmoidf_(g) * u);
   }
 }
 
 // one warp per (token, head); d <= 128
 template <typename T>
-__global__ void epi_qkv_linear_kernel(const float* C, int64_t ldc, int64_t M, int S, int nh, int d, float eps, T* q,
-                                      T* k, T* v, float* gl) {
+__global__ void epi_qkv_linear_kernel(CView C, int64_t M, int S, int nh, int d, float eps, T* q, T* k, T* v,
+                                      float* gl) {
   const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= M * nh) return;
   const int64_t r = w / nh;
   const int h = (int)(w % nh);
   const int64_t b = r / S, t = r % S;
-  const float* row = C + r * ldc;
   float sq = 0.f, sk = 0.f;
   for (int i = lane; i < d; i += 32) {
-    const float a = row[(int64_t)h * d + i], c = row[(int64_t)(nh + h) * d + i];
+    const float a = C(r, (int64_t)h * d + i), c = C(r, (int64_t)(nh + h) * d + i);
     sq += a * a;
     sk += c * c;
   }
@@ -119,17 +137,17 @@ __global__ void epi_qkv_linear_kernel(const float* C, int64_t ldc, int64_t M, in
   const float iq = rsqrtf(sq + eps), ik = rsqrtf(sk + eps);
   const int64_t o = ((b * nh + h) * S + t) * d;
   for (int i = lane; i < d; i += 32) {
-    q[o + i] = from_f<T>(row[(int64_t)h * d + i] * iq);
-    k[o + i] = from_f<T>(row[(int64_t)(nh + h) * d + i] * ik);
-    v[o + i] = from_f<T>(row[(int64_t)(2 * nh + h) * d + i]);
+    q[o + i] = from_f<T>(C(r, (int64_t)h * d + i) * iq);
+    k[o + i] = from_f<T>(C(r, (int64_t)(nh + h) * d + i) * ik);
+    v[o + i] = from_f<T>(C(r, (int64_t)(2 * nh + h) * d + i));
   }
-  if (lane == 0) gl[(b * nh + h) * S + t] = log_sigmoidf_(row[(int64_t)3 * nh * d + h]);
+  if (lane == 0) gl[(b * nh + h) * S + t] = log_sigmoidf_(C(r, (int64_t)3 * nh * d + h));
 }
 
 // one warp per (token, head) over q heads, then k heads, then v heads
 template <typename T>
-__global__ void epi_qkv_full_kernel(const float* C, int64_t ldc, int64_t M, int S, int nq, int nkv, int hd,
-                                    const float2* rope, const int32_t* start, int64_t ctx, T* q, T* K, T* V) {
+__global__ void epi_qkv_full_kernel(CView C, int64_t M, int S, int nq, int nkv, int hd, const float2* rope,
+                                    const int32_t* start, int64_t ctx, T* q, T* K, T* V) {
   const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int nheads = nq + 2 * nkv;
@@ -138,7 +156,7 @@ __global__ void epi_qkv_full_kernel(const float* C, int64_t ldc, int64_t M, int 
   const int h = (int)(w % nheads);
   const int64_t b = r / S, t = r % S;
   const int64_t pos = start[b] + t;
-  const float* src = C + r * ldc + (int64_t)h * hd;
+  const int64_t c0 = (int64_t)h * hd;
   const int half = hd / 2;
   T* dst;
   bool rot = true;
@@ -151,7 +169,7 @@ __global__ void epi_qkv_full_kernel(const float* C, int64_t ldc, int64_t M, int 
     rot = false;
   }
   for (int i = lane; i < half; i += 32) {
-    const float a = src[i], c = src[i + half];
+    const float a = C(r, c0 + i), c = C(r, c0 + i + half);
     if (rot) {
       const float2 cs = rope[pos * half + i];
       dst[i] = from_f<T>(a * cs.x - c * cs.y);
@@ -164,41 +182,43 @@ __global__ void epi_qkv_full_kernel(const float* C, int64_t ldc, int64_t M, int 
 }
 
 cudaError_t launch_epilogue_unfused(const float* C, int64_t ldc, int64_t M, int64_t N, const EpiArgs& e, bool bf,
-                                    cudaStream_t st) {
+                                    cudaStream_t st, int splits) {
   if (M == 0) return cudaSuccess;
   auto grid_for = [](int64_t n) { return (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 32); };
+  const CView cv{C, ldc, M * ldc, splits};
   switch (e.mode) {
     case Epi::F32:
+      if (splits > 1 || C != e.c) epi_f32_kernel<<<grid_for(M * N), 256, 0, st>>>(cv, M, N, e.c, e.ldc);
       break;
     case Epi::RESID:
-      epi_resid_kernel<<<grid_for(M * N), 256, 0, st>>>(C, ldc, M, N, e.c);
+      epi_resid_kernel<<<grid_for(M * N), 256, 0, st>>>(cv, M, N, e.c);
       break;
     case Epi::MHC_WRITE:
-      epi_mhc_kernel<<<grid_for(M * N), 256, 0, st>>>(C, ldc, M, N, e.s, e.coef);
+      epi_mhc_kernel<<<grid_for(M * N), 256, 0, st>>>(cv, M, N, e.s, e.coef);
       break;
     case Epi::SWIGLU:
-      if (bf) epi_swiglu_kernel<bf16><<<grid_for(M * N / 2), 256, 0, st>>>(C, ldc, M, N / 2, (bf16*)e.a);
-      else epi_swiglu_kernel<float><<<grid_for(M * N / 2), 256, 0, st>>>(C, ldc, M, N / 2, (float*)e.a);
+      if (bf) epi_swiglu_kernel<bf16><<<grid_for(M * N / 2), 256, 0, st>>>(cv, M, N / 2, (bf16*)e.a);
+      else epi_swiglu_kernel<float><<<grid_for(M * N / 2), 256, 0, st>>>(cv, M, N / 2, (float*)e.a);
       break;
     case Epi::QKV_LINEAR: {
       const int64_t warps = M * e.n_lin;
       const unsigned g = (unsigned)((warps * 32 + 255) / 256);
       if (bf)
-        epi_qkv_linear_kernel<bf16><<<g, 256, 0, st>>>(C, ldc, M, e.S, e.n_lin, e.hd, e.eps, (bf16*)e.q, (bf16*)e.k,
+        epi_qkv_linear_kernel<bf16><<<g, 256, 0, st>>>(cv, M, e.S, e.n_lin, e.hd, e.eps, (bf16*)e.q, (bf16*)e.k,
                                                        (bf16*)e.v, e.gl);
       else
-        epi_qkv_linear_kernel<float><<<g, 256, 0, st>>>(C, ldc, M, e.S, e.n_lin, e.hd, e.eps, (float*)e.q,
-                                                        (float*)e.k, (float*)e.v, e.gl);
+        epi_qkv_linear_kernel<float><<<g, 256, 0, st>>>(cv, M, e.S, e.n_lin, e.hd, e.eps, (float*)e.q, (float*)e.k,
+                                                        (float*)e.v, e.gl);
       break;
     }
     case Epi::QKV_FULL: {
       const int64_t warps = M * (e.heads_q + 2 * e.heads_kv);
       const unsigned g = (unsigned)((warps * 32 + 255) / 256);
       if (bf)
-        epi_qkv_full_kernel<bf16><<<g, 256, 0, st>>>(C, ldc, M, e.S, e.heads_q, e.heads_kv, e.hd, e.rope, e.start,
+        epi_qkv_full_kernel<bf16><<<g, 256, 0, st>>>(cv, M, e.S, e.heads_q, e.heads_kv, e.hd, e.rope, e.start,
                                                      e.cache_ctx, (bf16*)e.q, (bf16*)e.k, (bf16*)e.v);
       else
-        epi_qkv_full_kernel<float><<<g, 256, 0, st>>>(C, ldc, M, e.S, e.heads_q, e.heads_kv, e.hd, e.rope, e.start,
+        epi_qkv_full_kernel<float><<<g, 256, 0, st>>>(cv, M, e.S, e.heads_q, e.heads_kv, e.hd, e.rope, e.start,
                                                       e.cache_ctx, (float*)e.q, (float*)e.k, (float*)e.v);
       break;
     }

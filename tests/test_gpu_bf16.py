@@ -103,3 +103,43 @@ def test_mid_bf16_all_positions(B, S):
         assert L.loop_device_status() == 0
     finally:
         L.loop_model_destroy(g)
+
+
+MID4 = dict(MID, n_q=8, n_kv=2)  # GQA group 4 at head_dim 128: the decode-attention kernel's shape
+
+
+def test_mid_bf16_decode_matches_oracle():
+    """Prefill then decode steps on the tensor-core decode path (split-K
+    weight-streaming GEMM, chunked decode attention, GLA step)."""
+    B, S, steps = 3, 300, 4
+    m = dict(W.model_config("tiny_fp32", **MID4), max_batch=B, max_ctx=S + steps)
+    g = L.loop_model_create(L.make_config(**m), seed=6)
+    try:
+        o = oracle.Model(oracle.make_config(**m), seed=6)
+        tok = seeded.tokens(6, B, S, m["vocab"])
+        nxt = seeded.tokens(6, B, steps, m["vocab"], stream=seeded.S_DECODE_TOKENS)
+        ref = o.prefill(tok)
+        out = torch.empty((B, m["vocab"]), device="cuda")
+        L.loop_prefill(g, tokens=torch.from_numpy(tok).cuda(), out=out)
+        torch.cuda.synchronize()
+        check(out.cpu().numpy(), ref)
+        for t in range(steps):
+            r = o.decode_step(nxt[:, t])
+            L.loop_decode_step(g, torch.from_numpy(np.ascontiguousarray(nxt[:, t])).cuda(), out)
+            torch.cuda.synchronize()
+            check(out.cpu().numpy(), r)
+            assert L.loop_seq_len(g, 2) == o.seq_len(2) == S + t + 1
+        for slot in range(12):
+            st = torch.empty((B, 4, 128, 128), device="cuda")
+            L.loop_cache_read(g, L.LOOP_KIND_LINEAR, slot, B, 0, st)
+            torch.cuda.synchronize()
+            check(st.cpu().numpy(), o.state(slot, B))
+        kv = torch.empty((2, B, 2, S + steps, 128), device="cuda")
+        L.loop_cache_read(g, L.LOOP_KIND_FULL, 3, B, S + steps, kv)
+        k, v = o.kv(3, B, S + steps)
+        torch.cuda.synchronize()
+        check(kv[0].cpu().numpy(), k)
+        check(kv[1].cpu().numpy(), v)
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)

@@ -79,3 +79,41 @@ def test_loop9b_prefill_full_size():
     # floor; the cosine bound is the stated 0.999
     e, c = rel_err(got, ref), cosine(got, ref)
     assert e < noise_floor("loop9b_prefix16")["rel"] and c > COS_BF16, (e, c)
+
+
+def test_loop9b_decode_full_size():
+    """The decode workload: 64 sequences after a 32,768-token prefill, decoded
+    one token at a time.  A decode step must agree with a prefill of the
+    sequence one token longer (the prefill path is tied to the oracle above);
+    the sequence lengths advance exactly."""
+    w = W.WORKLOADS["loop9b_decode_b64_ctx32768"]
+    B, S = w["batch"], w["seq"]
+    m = dict(w["model"], max_batch=B, max_ctx=S + 4)
+    V = m["vocab"]
+    tok = seeded.tokens(w["seed"], B, S, V)
+    nxt = seeded.tokens(w["seed"], B, 2, V, stream=seeded.S_DECODE_TOKENS)
+    g = L.loop_model_create(L.make_config(**m), seed=w["seed"])
+    try:
+        out = torch.empty((B, V), device="cuda")
+        L.loop_prefill(g, tokens=torch.from_numpy(tok).cuda(), out=out)
+        d1 = torch.empty((B, V), device="cuda")
+        L.loop_decode_step(g, torch.from_numpy(nxt[:, 0].copy()).cuda(), d1)
+        d2 = torch.empty((B, V), device="cuda")
+        L.loop_decode_step(g, torch.from_numpy(nxt[:, 1].copy()).cuda(), d2)
+        torch.cuda.synchronize()
+        assert all(L.loop_seq_len(g, b) == S + 2 for b in (0, 17, 63))
+        assert torch.isfinite(d2).all()
+        got = {b: (d1[b].cpu().numpy(), d2[b].cpu().numpy()) for b in (0, 41)}
+        # reference: prefill of sequence b extended by its decode tokens
+        for b in (0, 41):
+            for i, gv in enumerate(got[b]):
+                ext = np.concatenate([tok[b], nxt[b, :i + 1]])[None].astype(np.int32)
+                ref = torch.empty((1, V), device="cuda")
+                L.loop_prefill(g, tokens=torch.from_numpy(ext).cuda(), out=ref)
+                torch.cuda.synchronize()
+                rv = ref[0].cpu().numpy()
+                e, c = rel_err(gv, rv), cosine(gv, rv)
+                assert e < noise_floor("loop9b_prefix16")["rel"] and c > COS_BF16, (b, i, e, c)
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
