@@ -156,6 +156,24 @@ LOOP_API int32_t mhc_prologue(const float* d_streams, int64_t T, int32_t H, cons
                               const float* d_phi, const float* d_gain, int32_t iters, float eps, float* d_coef,
                               void* d_xhat, int32_t xhat_dtype, float* d_scratch, void* stream);
 
+/* mhc_prologue for callers that cannot allocate device memory: code running
+ * under a framework or serving runtime whose memory pool owns every device
+ * allocation, or a latency-critical path that cannot afford the implicit
+ * synchronisation of cudaMalloc / cudaFree.  The pages have no counterpart;
+ * this is a calling convention of the library, not part of the method.
+ * Same arguments and results as mhc_prologue, without d_scratch: the scratch
+ * is a fixed array of 18 x 65,536 floats (4.7 MB) compiled into the library,
+ * which every GPU that loads the library holds until the process exits.
+ * Allocates nothing.  T > 65,536 returns LOOP_ERANGE.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  All calls
+ * on a device share the array and leave their values in it; calls that
+ * overlap on the GPU (for instance on two streams) race and must not be
+ * issued.  No part of the array needs to start at zero. */
+LOOP_API int32_t mhc_prologue_noalloc(const float* d_streams, int64_t T, int32_t H, const float* d_gamma,
+                                      const float* d_phi, const float* d_gain, int32_t iters, float eps,
+                                      float* d_coef, void* d_xhat, int32_t xhat_dtype, void* stream);
+
 /* Release everything the model owns.  Waits for the model's queued work. */
 LOOP_API void loop_model_destroy(loop_model* m);
 

@@ -25,7 +25,8 @@ KERNEL_CLASSES = ("gemm", "attention", "linear_attention", "mhc", "norm", "other
 API = ("loop_num_exec", "loop_schedule", "loop_num_weights", "loop_model_create", "loop_prefill",
        "loop_decode_step", "mhc_sinkhorn", "loop_model_destroy", "loop_seq_len", "loop_cache_read",
        "loop_weight_read", "loop_device_status", "loop_clear_device_status", "loop_last_error",
-       "loop_gemm_bf16", "loop_set_timing", "loop_timing_read", "loop_launch_count", "mhc_prologue")
+       "loop_gemm_bf16", "loop_set_timing", "loop_timing_read", "loop_launch_count", "mhc_prologue",
+       "mhc_prologue_noalloc")
 
 
 class loop_config(C.Structure):
@@ -80,6 +81,7 @@ def lib():
             "loop_timing_read": (i32, [vp, i32, P(C.c_double), P(C.c_int64), P(C.c_double), i32]),
             "loop_launch_count": (C.c_int64, [vp]),
             "mhc_prologue": (i32, [vp, C.c_int64, i32, vp, vp, vp, i32, C.c_float, vp, vp, i32, vp, vp]),
+            "mhc_prologue_noalloc": (i32, [vp, C.c_int64, i32, vp, vp, vp, i32, C.c_float, vp, vp, i32, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -222,3 +224,15 @@ def mhc_prologue(streams, gamma, phi, gain, coef, xhat, scratch, iters: int = 20
     dt = LOOP_BF16 if xhat.dtype == torch.bfloat16 else LOOP_F32
     _check("mhc_prologue", lib().mhc_prologue(_ptr(streams), T, H, _ptr(gamma), _ptr(phi), _ptr(gain), iters, eps,
                                               _ptr(coef), _ptr(xhat), dt, _ptr(scratch), _stream(stream)))
+
+
+def mhc_prologue_noalloc(streams, gamma, phi, gain, coef, xhat, iters: int = 20, eps: float = 1e-6,
+                         stream=None) -> None:
+    """mhc_prologue without a scratch argument: for callers that cannot
+    allocate device memory (the library's fixed scratch array is used)."""
+    import torch
+    T, H = int(streams.shape[1]), int(streams.shape[2])
+    dt = LOOP_BF16 if xhat.dtype == torch.bfloat16 else LOOP_F32
+    _check("mhc_prologue_noalloc", lib().mhc_prologue_noalloc(_ptr(streams), T, H, _ptr(gamma), _ptr(phi),
+                                                              _ptr(gain), iters, eps, _ptr(coef), _ptr(xhat), dt,
+                                                              _stream(stream)))

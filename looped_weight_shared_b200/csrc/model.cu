@@ -113,6 +113,8 @@ uint16_t bf16_bits_rne(float x) {
 
 bool bf16_model(const Model& m) { return m.c.dtype == LOOP_BF16; }
 
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+
 }  // namespace loopk
 
 using namespace loopk;

@@ -115,6 +115,9 @@ struct Model {
 
 bool bf16_model(const Model& m);
 
+// Record the text loop_last_error() returns on this thread.
+void set_last_error(const std::string& msg);
+
 // Device address of the library's status word (this device), or NULL.
 int* status_ptr();
 int status_read();
