@@ -41,6 +41,8 @@ def args_():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=12)
+    p.add_argument("--no-decode", action="store_true", help="skip the decode measurement of the default run")
+    p.add_argument("--decode-steps", type=int, default=32)
     return p.parse_args()
 
 
@@ -66,6 +68,34 @@ def metric_for(name, decode):
     if W.WORKLOADS[name]["model"]["io_mode"] == 1:
         return "looped 4-layer group prefill tokens/s at 9B width", "tokens/s"
     return "looped-decoder prefill tokens/s at 9B shape", "tokens/s"
+
+
+# ---------------------------------------------------------------------------- algorithmic work
+
+def layer_weight_bytes(m, full: bool) -> int:
+    H, F = m["hidden"], m["ffn"]
+    if full:
+        nq, nkv = m["n_q"] * m["head_dim"], m["n_kv"] * m["head_dim"]
+        w_in, w_o = (nq + 2 * nkv) * H, H * nq
+    else:
+        d = m["n_lin"] * m["lin_dim"]
+        w_in, w_o = (3 * d + m["n_lin"]) * H, H * d
+    return 2 * (w_in + w_o + 2 * F * H + H * F)
+
+
+def decode_step_bytes(m, B: int, ctx: int) -> dict:
+    """HBM bytes one decode step must move: every layer execution reads its
+    weights (the shared block twice), the head reads E, full attention reads
+    the KV cache of its slot, linear attention reads and writes its state."""
+    n_phys = m["n_prelude"] + m["n_block"] + m["n_coda"]
+    execs = list(range(m["n_prelude"])) + [m["n_prelude"] + j for j in range(m["n_block"])] * m["n_loops"] + \
+        [m["n_prelude"] + m["n_block"] + j for j in range(m["n_coda"])]
+    full = [p % m["group"] == m["full_slot"] for p in execs]
+    weights = sum(layer_weight_bytes(m, f) for f in full) + 2 * m["vocab"] * m["hidden"]
+    kv_row = m["n_kv"] * m["head_dim"] * 2 * 2
+    kv = sum(full) * B * (ctx + 1) * kv_row
+    state = (len(full) - sum(full)) * B * m["n_lin"] * m["lin_dim"] ** 2 * 4 * 2
+    return {"weights": weights, "kv": kv, "state": state, "total": weights + kv + state + sum(full) * B * kv_row}
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -251,6 +281,56 @@ def run_ours(a, rank, world, local_rank):
                 units=units)
 
 
+def run_decode(a, world, local_rank):
+    """Decode throughput: 64 sequences after a 32,768-token prefill."""
+    import torch
+    import looped_weight_shared_b200 as L
+
+    dev = torch.device("cuda", local_rank)
+    w = W.WORKLOADS["loop9b_decode_b64_ctx32768"]
+    m = dict(w["model"])
+    B, S, seed = w["batch"], w["seq"], w["seed"]
+    steps, warm = max(a.decode_steps, 1), max(a.warmup, 3)
+    m.update(max_batch=B, max_ctx=S + warm + steps + 2)
+    g = L.loop_model_create(L.make_config(**m), seed=seed)
+    V = m["vocab"]
+    out = torch.empty((B, V), device=dev)
+    L.loop_prefill(g, tokens=torch.from_numpy(seeded.tokens(seed, B, S, V)).to(dev), out=out)
+    nxt = seeded.tokens(seed, B, warm + steps, V, stream=seeded.S_DECODE_TOKENS)
+    toks = [torch.from_numpy(nxt[:, i].copy()).to(dev) for i in range(nxt.shape[1])]
+    for i in range(warm):
+        L.loop_decode_step(g, toks[i], out)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ctx0 = L.loop_seq_len(g, 0)
+    L.loop_timing_read(g, 0, reset=True)
+    L.loop_set_timing(g, True)
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        for i in range(steps):
+            L.loop_decode_step(g, toks[warm + i], out)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    L.loop_set_timing(g, False)
+    ms = ev0.elapsed_time(ev1) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    classes = {}
+    for ci, cname in enumerate(L.KERNEL_CLASSES):
+        tms, n, work = L.loop_timing_read(g, ci)
+        classes[cname] = {"ms_per_step": tms / steps, "launches": n}
+    L.loop_model_destroy(g)
+    mid_ctx = ctx0 + steps // 2
+    by = decode_step_bytes(m, B, mid_ctx)
+    return {"ms": ms, "value": B * world / (ms / 1e3), "bytes": by, "classes": classes, "clocks": clk.summary(),
+            "ctx": mid_ctx}
+
+
 # ---------------------------------------------------------------------------- oracle (CPU)
 
 def oracle_sample(a, steps=1):
@@ -348,6 +428,21 @@ def main():
             "gpu_launches": r["launches"],
             "kernel_ms_per_step": {k: round(v["ms_per_step"], 3) for k, v in r["classes"].items()},
             "device_status": r["status"]}
+    if a.workload == DEFAULT_WORKLOAD and not a.no_decode:
+        d = run_decode(a, world, local_rank)
+        kv_ms = d["classes"]["attention"]["ms_per_step"]
+        kv_gbs = d["bytes"]["kv"] / (kv_ms / 1e3) / 1e9 if kv_ms > 0 else 0.0
+        step_gbs = d["bytes"]["total"] / (d["ms"] / 1e3) / 1e9
+        line["decode"] = {
+            "metric": "looped-decoder decode tokens/s at 9B shape", "value": d["value"], "unit": "tokens/s",
+            "ms_per_step": d["ms"], "workload": "loop9b_decode_b64_ctx32768", "batch": 64, "context": d["ctx"],
+            "bytes_per_step": d["bytes"],
+            "step_roofline": {"bound": "hbm", "achieved": step_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                              "frac": step_gbs / pk["hbm_gbs"], "peak_kind": f"{pk_kind} copy bandwidth"},
+            "roofline": {"bound": "hbm", "kernel": "decode attention (KV-cache read)", "achieved": kv_gbs,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": kv_gbs / pk["hbm_gbs"], "traffic": None},
+            "kernel_ms_per_step": {k: round(v["ms_per_step"], 3) for k, v in d["classes"].items()},
+            "clocks": d["clocks"]}
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         c = oracle_sample(a, steps=1)
         line["cpu_baseline"] = {"value": c["value"], "unit": unit, "cores": c["cores"], "kind": "oracle",

@@ -220,10 +220,11 @@ cudaError_t launch_sinkhorn(const float* l, float* out, int64_t count, int n, in
 // mHC prologue for n = 2 streams, in two HBM-streaming kernels.
 //
 // (A) mhc_partial: the flattened stream vector u = (s_0, s_1) of a token has
-//     2H entries; CTA (blk, half) keeps half of Phi and gamma (H entries each,
-//     fp32, 8 x H + H floats) in shared memory and every warp streams 8 tokens
-//     of that half with float4 loads, so each Phi value read is used 8 times.
-//     It writes, per token and half, the 8 partial projections
+//     2H entries, cut into `parts` equal parts (2 for long inputs; more when
+//     few tokens must still spread over many SMs); CTA (blk, part) keeps its
+//     part of Phi and gamma in shared memory and every warp streams 8 tokens
+//     of that part with float4 loads, so each Phi value read is used 8 times.
+//     It writes, per token and part, the 8 partial projections
 //     sum_i s_i gamma_i Phi_ci and the partial sum of squares.
 // (B) mhc_read: one warp per token folds the two halves into
 //     l = (sum / r), r = sqrt(sum of squares / 2H + eps), forms H_pre, H_post
@@ -237,39 +238,41 @@ constexpr int MHCB_WARPS = 8;
 
 __global__ void __launch_bounds__(MHCA_THREADS, 1)
     mhc_partial_kernel(const float* __restrict__ s, int64_t T, int H, const float* __restrict__ gamma,
-                       const float* __restrict__ phi, float* __restrict__ part) {
+                       const float* __restrict__ phi, int parts, float* __restrict__ part) {
   extern __shared__ float4 sm4[];
-  const int half = blockIdx.y;
-  const int H4 = H / 4, D = 2 * H;
-  float4* sphi = sm4;            // [8][H4]
-  float4* sgam = sm4 + 8 * H4;   // [H4]
-  for (int i = threadIdx.x; i < H4; i += MHCA_THREADS) {
+  const int p = blockIdx.y;
+  const int D = 2 * H, PL = D / parts, PL4 = PL / 4;
+  const int i0 = p * PL;                  // this part's first entry of the flattened streams
+  const int stream = i0 / H, col0 = i0 % H;  // a part lies inside one stream
+  float4* sphi = sm4;             // [8][PL4]
+  float4* sgam = sm4 + 8 * PL4;   // [PL4]
+  for (int i = threadIdx.x; i < PL4; i += MHCA_THREADS) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      sphi[c * H4 + i] = reinterpret_cast<const float4*>(phi + (int64_t)c * D + (int64_t)half * H)[i];
-    sgam[i] = reinterpret_cast<const float4*>(gamma + (int64_t)half * H)[i];
+    for (int c = 0; c < 8; ++c) sphi[c * PL4 + i] = reinterpret_cast<const float4*>(phi + (int64_t)c * D + i0)[i];
+    sgam[i] = reinterpret_cast<const float4*>(gamma + i0)[i];
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t0 = ((int64_t)blockIdx.x * MHCA_WARPS + warp) * MHCA_TOK;
   if (t0 >= T) return;
   const int ntok = (int)(T - t0 < MHCA_TOK ? T - t0 : MHCA_TOK);
-  const float4* base = reinterpret_cast<const float4*>(s + ((int64_t)half * T + t0) * H);
+  const int H4 = H / 4;
+  const float4* base = reinterpret_cast<const float4*>(s + ((int64_t)stream * T + t0) * H + col0);
   float acc[MHCA_TOK][9];
 #pragma unroll
   for (int j = 0; j < MHCA_TOK; ++j)
 #pragma unroll
     for (int c = 0; c < 9; ++c) acc[j][c] = 0.f;
 #pragma unroll 2
-  for (int f = lane; f < H4; f += 32) {
+  for (int f = lane; f < PL4; f += 32) {
     float4 v[MHCA_TOK];
 #pragma unroll
     for (int j = 0; j < MHCA_TOK; ++j) v[j] = j < ntok ? __ldcs(base + (int64_t)j * H4 + f) : make_float4(0, 0, 0, 0);
     const float4 g = sgam[f];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      const float4 p = sphi[c * H4 + f];
-      const float4 w = make_float4(p.x * g.x, p.y * g.y, p.z * g.z, p.w * g.w);
+      const float4 ph = sphi[c * PL4 + f];
+      const float4 w = make_float4(ph.x * g.x, ph.y * g.y, ph.z * g.z, ph.w * g.w);
 #pragma unroll
       for (int j = 0; j < MHCA_TOK; ++j) acc[j][c] += v[j].x * w.x + v[j].y * w.y + v[j].z * w.z + v[j].w * w.w;
     }
@@ -281,21 +284,24 @@ __global__ void __launch_bounds__(MHCA_THREADS, 1)
 #pragma unroll
     for (int c = 0; c < 9; ++c) {
       const float r = warp_sum(acc[j][c]);
-      if (lane == c && j < ntok) part[((t0 + j) * 2 + half) * 9 + c] = r;
+      if (lane == c && j < ntok) part[((t0 + j) * parts + p) * 9 + c] = r;
     }
 }
 
 template <typename T>
 __global__ void __launch_bounds__(MHCB_WARPS * 32)
-    mhc_read_kernel(const float* __restrict__ s, int64_t Ttot, int H, const float* __restrict__ part,
+    mhc_read_kernel(const float* __restrict__ s, int64_t Ttot, int H, const float* __restrict__ part, int parts,
                     const float* __restrict__ gain, int iters, float eps, float* __restrict__ coef, T* __restrict__ xh) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * MHCB_WARPS + warp;
   if (t >= Ttot) return;
-  const float* pp = part + t * 18;
+  const float* pp = part + t * parts * 9;
   float tot[9];
 #pragma unroll
-  for (int c = 0; c < 9; ++c) tot[c] = pp[c] + pp[9 + c];
+  for (int c = 0; c < 9; ++c) tot[c] = pp[c];
+  for (int q = 1; q < parts; ++q)
+#pragma unroll
+    for (int c = 0; c < 9; ++c) tot[c] += pp[q * 9 + c];
   const float rinv = rsqrtf(tot[8] / (2 * H) + eps);
   float l[8];
 #pragma unroll
@@ -342,20 +348,24 @@ size_t mhc_partial_smem(int H) { return (size_t)9 * H * sizeof(float); }
 
 cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf,
-                                float* part, cudaStream_t st) {
+                                float* part, cudaStream_t st, int parts) {
   if (T == 0) return cudaSuccess;
   if (H % 4 != 0 || mhc_partial_smem(H) > 220 * 1024) return cudaErrorInvalidValue;
-  const int smem = (int)mhc_partial_smem(H);
-  cudaError_t e = cudaFuncSetAttribute(mhc_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (parts < 2 || parts % 2 != 0 || (2 * H) % (4 * parts) != 0 || H % (2 * H / parts) != 0)
+    return cudaErrorInvalidValue;
+  const int smem = (int)(mhc_partial_smem(H) * 2 / parts);
+  cudaError_t e = cudaFuncSetAttribute(mhc_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)mhc_partial_smem(H));
   if (e != cudaSuccess) return e;
   const int64_t per_cta = (int64_t)MHCA_WARPS * MHCA_TOK;
-  dim3 ga((unsigned)((T + per_cta - 1) / per_cta), 2);
-  mhc_partial_kernel<<<ga, MHCA_THREADS, smem, st>>>(s, T, H, gamma, phi, part);
+  dim3 ga((unsigned)((T + per_cta - 1) / per_cta), (unsigned)parts);
+  mhc_partial_kernel<<<ga, MHCA_THREADS, smem, st>>>(s, T, H, gamma, phi, parts, part);
   const unsigned gb = (unsigned)((T + MHCB_WARPS - 1) / MHCB_WARPS);
   if (bf)
-    mhc_read_kernel<bf16><<<gb, MHCB_WARPS * 32, 0, st>>>(s, T, H, part, gain, iters, eps, coef, (bf16*)xh);
+    mhc_read_kernel<bf16><<<gb, MHCB_WARPS * 32, 0, st>>>(s, T, H, part, parts, gain, iters, eps, coef, (bf16*)xh);
   else
-    mhc_read_kernel<float><<<gb, MHCB_WARPS * 32, 0, st>>>(s, T, H, part, gain, iters, eps, coef, (float*)xh);
+    mhc_read_kernel<float><<<gb, MHCB_WARPS * 32, 0, st>>>(s, T, H, part, parts, gain, iters, eps, coef,
+                                                           (float*)xh);
   return cudaGetLastError();
 }
 

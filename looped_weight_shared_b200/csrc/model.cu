@@ -315,7 +315,8 @@ int32_t create_impl(const loop_config* cfg, const float* const* hw, uint64_t see
   LOOP_ALLOC(w.s, float*, 2 * T * H * 4);
   LOOP_ALLOC(w.xh, void*, T * H * es);
   LOOP_ALLOC(w.coef, float*, T * 8 * 4);
-  LOOP_ALLOC(w.mhc_part, float*, T * 18 * 4);
+  w.mhc_part_floats = std::max<int64_t>(T * 18, 512 * 16 * 9);
+  LOOP_ALLOC(w.mhc_part, float*, w.mhc_part_floats * 4);
   if (m.use_tc && H % 64 == 0) {  // decode GEMM partials: up to 32 splits x 64 tokens x the widest projection
     int64_t maxn = std::max<int64_t>(2 * F, H);
     for (auto& L : m.L) maxn = std::max(maxn, L.n_in);
@@ -514,9 +515,12 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
       const float* gain = sub == 0 ? L.attn_gain : L.ffn_gain;
       if (in_block) {
         const SiteW& site = m.sites[2 * (phys - c.n_prelude) + sub];
+        // decode (few tokens): cut Phi into 16 parts so the partial kernel spreads over the SMs;
+        // a prefill always uses 2, so each row's arithmetic is the same at any length
+        const int parts = (m.decoding && H % 32 == 0 && T * 16 * 9 <= w.mhc_part_floats) ? 16 : 2;
         LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), 2, st, [&] {
           return launch_mhc_prologue(s_buf, T, (int)H, site.gamma, site.phi, gain, c.sinkhorn_iters, c.norm_eps,
-                                     w.coef, w.xh, bf, w.mhc_part, st);
+                                     w.coef, w.xh, bf, w.mhc_part, st, parts);
         }));
       } else {
         LOOP_CU(timed(m, LOOP_K_NORM, (double)T * H * (4 + es), 1, st,

@@ -73,7 +73,8 @@ struct Work {
   float* cbuf = nullptr;    // [T][max N] projection scratch of the unfused path
   void* xf = nullptr;       // [rows][H] final-norm output
   int32_t* zeros = nullptr; // start positions of a prefill (all 0)
-  float* mhc_part = nullptr;  // [T][2][9] partial projections of the mHC prologue
+  float* mhc_part = nullptr;  // [T][parts][9] partial projections of the mHC prologue
+  int64_t mhc_part_floats = 0;
   float* cpart = nullptr;     // split-K partial sums of the decode GEMM [32][64][max N]
   int64_t cpart_floats = 0;
   float* dec_attn = nullptr;  // decode attention chunk partials [B][n_q][ctx / 128][130]
@@ -131,10 +132,11 @@ cudaError_t launch_embed(const int32_t* tok, const void* E, bool bf16, int64_t T
                          cudaStream_t st);
 cudaError_t launch_rmsnorm(const float* x, int64_t rows, int H, int64_t row_step, int64_t row_off,
                            const float* gain, float eps, void* y, bool bf16, cudaStream_t st);
-// two kernels; `part` is scratch of 18 floats per token
+// two kernels; `part` is scratch of 9 x parts floats per token (parts even,
+// dividing the stream width into equal float4 runs; 2 by default)
 cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf16,
-                                float* part, cudaStream_t st);
+                                float* part, cudaStream_t st, int parts = 2);
 size_t mhc_partial_smem(int H);
 cudaError_t launch_expand(const float* h, float* s, int64_t n, cudaStream_t st);
 cudaError_t launch_collapse(const float* s, float* h, int64_t n, cudaStream_t st);

@@ -36,6 +36,9 @@ WORKLOADS = {
     "loop9b_decode_b64_ctx32768": dict(model=_LOOP9B, batch=64, seq=32768, seed=3, decode_steps=128),
     # the 9B-shaped looped decoder, one 262,144-token prefill
     "loop9b_prefill_b1_s262144": dict(model=_LOOP9B, batch=1, seq=262144, seed=4),
+    # small probes for kernel captures (9B kernel shapes, a few GB on the device)
+    "probe_decode_b64_ctx4096": dict(model=dict(_GROUP9B, vocab=4096, io_mode=0), batch=64, seq=4096, seed=3,
+                                     decode_steps=16),
 }
 
 
