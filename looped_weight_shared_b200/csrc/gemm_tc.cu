@@ -9,9 +9,10 @@
 //   warp 1      one thread issues tcgen05.mma (M = 128, N = 256, K = 16) into
 //               one of two 256-column TMEM accumulators;
 //   warp 2      allocates / frees the 512 TMEM columns;
-//   warps 4-7   epilogue: tcgen05.ld of the accumulator rows (warp w reads
-//               TMEM lanes 32 (w % 4) ..), fused output, then release the
-//               accumulator so the next tile's MMAs overlap this epilogue.
+//   warps 4-11  epilogue, two warpgroups splitting the tile's columns:
+//               tcgen05.ld of the accumulator rows (warp w reads TMEM lanes
+//               32 (w % 4) ..), fused output, then release the accumulator
+//               so the next tile's MMAs overlap this epilogue.
 // Every wait on an mbarrier gives up after ~2 s and flags the status word.
 
 #include <cuda.h>
@@ -31,7 +32,8 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-constexpr int THREADS = 256;
+constexpr int THREADS = 256;       // skinny kernel: 4 role warps + 4 epilogue warps
+constexpr int GEMM_THREADS = 384;  // main kernel: 4 role warps + 8 epilogue warps (two column halves)
 constexpr int TMEM_COLS = 512;
 constexpr int GROUP_M = 16;  // tile raster: GROUP_M row blocks sweep the N blocks together
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
@@ -116,12 +118,14 @@ LOOP_DEV void head_store_rope(uint32_t t0, bf16* dst, const float2* cs_row, bool
 
 // tcgen05.ld / wait::ld are warp-collective: every lane of the warp executes
 // them in lockstep, and only the memory accesses of rows >= M are skipped.
+// Two epilogue warpgroups share a tile: `half` 0 takes the first 128
+// columns (or the first head, or gate/up chunks 0-1), `half` 1 the rest.
 template <Epi MODE>
-LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, const EpiP& p) {
+LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, int half, const EpiP& p) {
   const bool valid = row < p.M;
   if constexpr (MODE == Epi::F32) {
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = 4 * half; c < 4 * half + 4; ++c) {
       const int n = n0 + 32 * c;
       if (n >= p.N) break;
       float v[32];
@@ -138,7 +142,7 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, const EpiP& p) {
     }
   } else if constexpr (MODE == Epi::RESID) {
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = 4 * half; c < 4 * half + 4; ++c) {
       const int n = n0 + 32 * c;
       float v[32];
       ld_chunk(tacc + 32 * c, v);
@@ -160,7 +164,7 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, const EpiP& p) {
     // c0 = (pre0, pre1, post0, post1), c1 = (res00, res01, res10, res11)
     const int64_t plane = (int64_t)p.M * p.N;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = 4 * half; c < 4 * half + 4; ++c) {
       const int n = n0 + 32 * c;
       float v[32];
       ld_chunk(tacc + 32 * c, v);
@@ -196,7 +200,7 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, const EpiP& p) {
     const int F = p.N / 2;
     bf16* dst = p.a + (int64_t)row * F + n0 / 2;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 2 * half; c < 2 * half + 2; ++c) {
       float g[32], u[32];
       ld_chunk(tacc + 32 * c, g);
       ld_chunk(tacc + 128 + 32 * c, u);
@@ -211,13 +215,10 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, const EpiP& p) {
     const int region = n0 / (nl * d);  // 0 q, 1 k, 2 v, 3 gate
     if (region < 3) {
       bf16* base = region == 0 ? p.q : (region == 1 ? p.k : p.v);
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        const int head = (n0 - region * nl * d) / d + hh;
-        bf16* dst = base + (((int64_t)b * nl + head) * p.S + t) * d;
-        head_store(tacc + 128 * hh, dst, region < 2, p.eps, valid);
-      }
-    } else {
+      const int head = (n0 - region * nl * d) / d + half;
+      bf16* dst = base + (((int64_t)b * nl + head) * p.S + t) * d;
+      head_store(tacc + 128 * half, dst, region < 2, p.eps, valid);
+    } else if (half == 0) {
       float v[32];
 #pragma unroll 1
       for (int c = 0; c * 32 < nl; ++c) {
@@ -235,10 +236,9 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, const EpiP& p) {
     const int b = row / p.S, t = row % p.S;
     const int64_t pos = valid ? p.start[b] + t : 0;
     const float2* cs = p.rope + pos * (d / 2);
-#pragma unroll 1
-    for (int hh = 0; hh < 2; ++hh) {
-      const int head = n0 / d + hh;
-      const uint32_t t0 = tacc + 128 * hh;
+    {
+      const int head = n0 / d + half;
+      const uint32_t t0 = tacc + 128 * half;
       if (head < p.hq) {
         head_store_rope(t0, p.q + (((int64_t)b * p.hq + head) * p.S + t) * d, cs, valid);
       } else if (head < p.hq + p.hkv) {
@@ -262,7 +262,7 @@ LOOP_DEV void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
 }
 
 template <Epi MODE>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb, int M, int N,
                    int K, EpiP p, int* status) {
   extern __shared__ uint8_t smem_raw[];
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 8);  // one arrival per epilogue warp
     }
     fence_mbar_init();
   }
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, got)) break;  // the whole warp leaves together
       tc_fence_after();
       const uint32_t tacc = tmem + acc * BN + ((uint32_t)(32 * q) << 16);
-      epilogue_tile<MODE>(tacc, mb * BM + 32 * q + lane, nb * BN, p);
+      epilogue_tile<MODE>(tacc, mb * BM + 32 * q + lane, nb * BN, (warp - 4) >> 2, p);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -513,7 +513,7 @@ cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, int M, int
   }
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = std::min(tiles, num_sms());
-  gemm_tc_kernel<MODE><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, M, N, K, p, status_ptr());
+  gemm_tc_kernel<MODE><<<grid, GEMM_THREADS, SMEM_BYTES, st>>>(ma, mb, M, N, K, p, status_ptr());
   return cudaGetLastError();
 }
 
@@ -523,7 +523,7 @@ bool gemm_skinny_supported(int64_t M, int64_t N, int64_t K) { return M >= 1 && M
 
 int gemm_skinny_splits(int64_t N, int64_t K) {
   const int64_t tiles = (N + BM - 1) / BM, kbs = K / BK;
-  int64_t s = (2 * (int64_t)num_sms() + tiles - 1) / tiles;
+  int64_t s = (2 * (int64_t)num_sms() + tiles - 1) / tiles;  // about two waves of CTAs
   return (int)std::max<int64_t>(1, std::min<int64_t>({s, kbs, 32}));
 }
 

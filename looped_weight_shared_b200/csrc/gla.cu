@@ -298,9 +298,65 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// One decode step of gated linear attention (d = 128): S = g S + k v^T,
+// o = q S.  CTA (32-column slice of S, head, sequence), 256 threads: thread
+// (row group rg = tid / 32, column c = tid % 32) updates rows 16 rg .. 16 rg + 15
+// of its column with 16 independent loads, and the 8 row groups' parts of
+// q S are summed in shared memory.  The state is read and written once.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    gla_decode_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+                      const float* __restrict__ gl, float* __restrict__ state, bf16* __restrict__ out, int nh) {
+  __shared__ float qs[DK], ks[DK], red[8][32];
+  const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, rg = tid >> 5, c = tid & 31;
+  const int64_t bh = (int64_t)b * nh + h;
+  if (tid < DK) {
+    qs[tid] = __bfloat162float(q[bh * DK + tid]);
+    ks[tid] = __bfloat162float(k[bh * DK + tid]);
+  }
+  __syncthreads();
+  const int col = slice * 32 + c;
+  const float g = __expf(gl[bh]);
+  const float vc = __bfloat162float(v[bh * DK + col]);
+  float* st = state + bh * DK * 128 + col;
+  float sv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) sv[i] = st[(int64_t)(rg * 16 + i) * 128];
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = rg * 16 + i;
+    sv[i] = g * sv[i] + ks[r] * vc;
+    acc += qs[r] * sv[i];
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) st[(int64_t)(rg * 16 + i) * 128] = sv[i];
+  red[rg][c] = acc;
+  __syncthreads();
+  if (rg == 0) {
+    float o = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o += red[j][c];
+    out[(int64_t)b * nh * 128 + h * 128 + col] = __float2bfloat16_rn(o);
+  }
+}
+
 }  // namespace
 
 bool gla_chunk_supported(int d) { return d == DK; }
+
+// q, k, v [B][nh][1][128] bf16; gl [B][nh]; state [B][nh][128][128] fp32
+// (updated in place); o [B][nh * 128] bf16.
+cudaError_t launch_gla_decode(const void* q, const void* k, const void* v, const float* gl, float* state, void* o,
+                              int B, int nh, cudaStream_t st) {
+  if (B == 0) return cudaSuccess;
+  dim3 grid(128 / 32, (unsigned)nh, (unsigned)B);
+  gla_decode_kernel<<<grid, 256, 0, st>>>((const bf16*)q, (const bf16*)k, (const bf16*)v, gl, state, (bf16*)o, nh);
+  return cudaGetLastError();
+}
 
 // q, k, v [B][nh][S][128] bf16; gl [B][nh][S] log-gates; state [B][nh][128][128]
 // fp32 (read, then replaced by the final state); o [B*S][nh*128] bf16.

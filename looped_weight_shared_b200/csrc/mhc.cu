@@ -344,6 +344,73 @@ __global__ void __launch_bounds__(MHCB_WARPS * 32)
   }
 }
 
+// One-pass reader for H = 512 * NPL: one 128-thread CTA per token, each
+// thread keeps its NPL float4 of both streams in registers (loads issued
+// first), one lane forms the coefficients while those loads are in flight.
+template <typename T, int NPL>
+__global__ void __launch_bounds__(128)
+    mhc_read1_kernel(const float* __restrict__ s, int64_t Ttot, const float* __restrict__ part, int parts,
+                     const float* __restrict__ gain, int iters, float eps, float* __restrict__ coef,
+                     T* __restrict__ xh) {
+  constexpr int H = 512 * NPL;
+  __shared__ float cf[2];
+  __shared__ float red[4];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t = blockIdx.x;
+  const float4* s0 = reinterpret_cast<const float4*>(s + t * H);
+  const float4* s1 = reinterpret_cast<const float4*>(s + (Ttot + t) * H);
+  float4 a[NPL], b[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) a[i] = __ldcs(s0 + tid + 128 * i);
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) b[i] = __ldcs(s1 + tid + 128 * i);
+  if (tid == 0) {
+    const float* pp = part + t * parts * 9;
+    float tot[9];
+    for (int c = 0; c < 9; ++c) tot[c] = pp[c];
+    for (int q = 1; q < parts; ++q)
+      for (int c = 0; c < 9; ++c) tot[c] += pp[q * 9 + c];
+    const float rinv = rsqrtf(tot[8] / (2 * H) + eps);
+    float l[8];
+    for (int c = 0; c < 8; ++c) l[c] = tot[c] * rinv;
+    float P[4];
+    sinkhorn_fixed<2>(l + 4, P, iters);
+    const float pre0 = sigmoidf_(l[0]), pre1 = sigmoidf_(l[1]);
+    cf[0] = pre0;
+    cf[1] = pre1;
+    float4* co = reinterpret_cast<float4*>(coef + t * 8);
+    co[0] = make_float4(pre0, pre1, 2.f * sigmoidf_(l[2]), 2.f * sigmoidf_(l[3]));
+    co[1] = make_float4(P[0], P[1], P[2], P[3]);
+  }
+  __syncthreads();
+  const float pre0 = cf[0], pre1 = cf[1];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    a[i] = make_float4(pre0 * a[i].x + pre1 * b[i].x, pre0 * a[i].y + pre1 * b[i].y, pre0 * a[i].z + pre1 * b[i].z,
+                       pre0 * a[i].w + pre1 * b[i].w);
+    ss += a[i].x * a[i].x + a[i].y * a[i].y + a[i].z * a[i].z + a[i].w * a[i].w;
+  }
+  ss = warp_sum(ss);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  const float nrm = rsqrtf((red[0] + red[1] + red[2] + red[3]) / H + eps);
+  const float4* g4 = reinterpret_cast<const float4*>(gain);
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const float4 g = g4[tid + 128 * i];
+    const float x0 = a[i].x * nrm * g.x, x1 = a[i].y * nrm * g.y, x2 = a[i].z * nrm * g.z, x3 = a[i].w * nrm * g.w;
+    if constexpr (sizeof(T) == 2) {
+      uint2 u;
+      u.x = pack_bf16x2(x0, x1);
+      u.y = pack_bf16x2(x2, x3);
+      reinterpret_cast<uint2*>(xh + t * H)[tid + 128 * i] = u;
+    } else {
+      reinterpret_cast<float4*>(xh + t * H)[tid + 128 * i] = make_float4(x0, x1, x2, x3);
+    }
+  }
+}
+
 size_t mhc_partial_smem(int H) { return (size_t)9 * H * sizeof(float); }
 
 cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,
@@ -360,6 +427,11 @@ cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* g
   const int64_t per_cta = (int64_t)MHCA_WARPS * MHCA_TOK;
   dim3 ga((unsigned)((T + per_cta - 1) / per_cta), (unsigned)parts);
   mhc_partial_kernel<<<ga, MHCA_THREADS, smem, st>>>(s, T, H, gamma, phi, parts, part);
+  if (H == 4096) {  // the 9B width: one pass over the streams
+    if (bf) mhc_read1_kernel<bf16, 8><<<(unsigned)T, 128, 0, st>>>(s, T, part, parts, gain, iters, eps, coef, (bf16*)xh);
+    else mhc_read1_kernel<float, 8><<<(unsigned)T, 128, 0, st>>>(s, T, part, parts, gain, iters, eps, coef, (float*)xh);
+    return cudaGetLastError();
+  }
   const unsigned gb = (unsigned)((T + MHCB_WARPS - 1) / MHCB_WARPS);
   if (bf)
     mhc_read_kernel<bf16><<<gb, MHCB_WARPS * 32, 0, st>>>(s, T, H, part, parts, gain, iters, eps, coef, (bf16*)xh);

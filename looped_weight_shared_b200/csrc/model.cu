@@ -483,6 +483,10 @@ cudaError_t linear_attention(Model& m, float* state, int B, int S, cudaStream_t 
     });
   }
   const double flops = 4.0 * (double)B * S * c.n_lin * d * d;
+  if (bf && S == 1 && gla_chunk_supported(c.lin_dim))
+    return timed(m, LOOP_K_LINEAR_ATTENTION, flops, 1, st, [&] {
+      return launch_gla_decode(m.w.q, m.w.k, m.w.v, m.w.gl, state, m.w.o, B, c.n_lin, st);
+    });
   return timed(m, LOOP_K_LINEAR_ATTENTION, flops, 1, st, [&] {
     return launch_gla_recurrent(m.w.q, m.w.k, m.w.v, m.w.gl, state, m.w.o, bf, B, S, c.n_lin, c.lin_dim, st);
   });

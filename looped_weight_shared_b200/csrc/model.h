@@ -176,6 +176,10 @@ bool gla_chunk_supported(int d);
 cudaError_t launch_gla_chunked(const void* q, const void* k, const void* v, const float* gl, float* state, void* o,
                                int B, int S, int nh, cudaStream_t st);
 
+// one decode step of gated linear attention (bf16, d = 128)
+cudaError_t launch_gla_decode(const void* q, const void* k, const void* v, const float* gl, float* state, void* o,
+                              int B, int nh, cudaStream_t st);
+
 // tcgen05 GEMM (bf16): C = A[M][K] W[N][K]^T with a fused epilogue.  Returns
 // cudaErrorNotSupported when the shapes are outside what it handles.
 cudaError_t launch_gemm_tc(const void* A, const void* W, int64_t M, int64_t N, int64_t K, const EpiArgs& e,

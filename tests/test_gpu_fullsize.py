@@ -117,3 +117,43 @@ def test_loop9b_decode_full_size():
         assert L.loop_device_status() == 0
     finally:
         L.loop_model_destroy(g)
+
+
+def test_loop9b_long_prefill_full_size():
+    """The long-context workload: one 262,144-token prefill of the 9B-shaped
+    model.  Keys and values at a position depend only on the tokens up to it,
+    so the first rows of every full-attention execution's KV slot after the
+    long prefill are bit-identical to those of a short prefill of the prefix,
+    and that short prefill's logits agree with the oracle."""
+    w = W.WORKLOADS["loop9b_prefill_b1_s262144"]
+    S, P = w["seq"], 16
+    m = dict(w["model"], max_batch=1, max_ctx=S)
+    V = m["vocab"]
+    tok = seeded.tokens(w["seed"], 1, S, V)
+    g = L.loop_model_create(L.make_config(**m), seed=w["seed"])
+    try:
+        out = torch.empty((1, V), device="cuda")
+        L.loop_prefill(g, tokens=torch.from_numpy(tok).cuda(), out=out)
+        torch.cuda.synchronize()
+        assert torch.isfinite(out).all() and L.loop_seq_len(g, 0) == S
+        long_kv = []
+        for slot in range(14):
+            kv = torch.empty((2, 1, 8, P, 128), device="cuda")
+            L.loop_cache_read(g, L.LOOP_KIND_FULL, slot, 1, P, kv)
+            long_kv.append(kv)
+        short = torch.empty((1, P, V), device="cuda")
+        L.loop_prefill(g, tokens=torch.from_numpy(tok[:, :P].copy()).cuda(), out=short, flags=L.LOOP_ALL_POSITIONS)
+        for slot in range(14):
+            kv = torch.empty((2, 1, 8, P, 128), device="cuda")
+            L.loop_cache_read(g, L.LOOP_KIND_FULL, slot, 1, P, kv)
+            torch.cuda.synchronize()
+            assert torch.equal(kv, long_kv[slot]), slot
+        got = short[0].cpu().numpy()
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
+    o = oracle.Model(oracle.make_config(**dict(m, max_ctx=P)), seed=w["seed"])
+    ref = o.prefill(tok[:, :P], all_positions=True)[0]
+    o.close()
+    e, c = rel_err(got, ref), cosine(got, ref)
+    assert e < noise_floor("loop9b_prefix16")["rel"] and c > COS_BF16, (e, c)
