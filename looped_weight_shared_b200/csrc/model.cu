@@ -461,9 +461,9 @@ cudaError_t attention(Model& m, const void* Kc, const void* Vc, int B, int S, co
                                      m.w.dec_attn, st);
     });
   }
-  if (bf && S > 1 && flash_supported(c.head_dim, c.n_q, c.n_kv))  // a prefill: every sequence starts at 0
+  if (bf && S > 1 && flash_tc_supported(c.head_dim, c.n_q, c.n_kv))  // a prefill: every sequence starts at 0
     return timed(m, LOOP_K_ATTENTION, flops, 1, st, [&] {
-      return launch_flash_prefill(m.w.q, Kc, Vc, m.w.o, B, S, c.n_q, c.n_kv, c.max_ctx, st);
+      return launch_flash_tc(m.w.q, Kc, Vc, m.w.o, B, S, c.n_q, c.n_kv, c.max_ctx, st);
     });
   return timed(m, LOOP_K_ATTENTION, flops, 1, st, [&] {
     return launch_attention_simple(m.w.q, Kc, Vc, m.w.o, bf, B, S, c.n_q, c.n_kv, c.head_dim, c.max_ctx, d_start, st);

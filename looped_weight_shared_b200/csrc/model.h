@@ -160,10 +160,10 @@ cudaError_t launch_set_len(int32_t* seq_len, int B, int S, cudaStream_t st);
 cudaError_t launch_weight_to_f32(const void* src, bool bf16, int64_t rows, int64_t cols, int64_t src_row0,
                                  float* dst, cudaStream_t st);
 
-// flash attention for prefill (bf16, head_dim 128, all sequences from position 0)
-bool flash_supported(int hd, int nq, int nkv);
-cudaError_t launch_flash_prefill(const void* q, const void* K, const void* V, void* o, int B, int S, int nq, int nkv,
-                                 int64_t ctx, cudaStream_t st);
+// flash attention for prefill on tcgen05 (bf16, head_dim 128, all sequences from position 0)
+bool flash_tc_supported(int hd, int nq, int nkv);
+cudaError_t launch_flash_tc(const void* q, const void* K, const void* V, void* o, int B, int S, int nq, int nkv,
+                            int64_t ctx, cudaStream_t st);
 
 // decode attention (flash-decoding over 128-key chunks; bf16, head_dim 128, group 4)
 bool decode_attention_supported(int hd, int nq, int nkv);
