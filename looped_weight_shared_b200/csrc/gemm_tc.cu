@@ -368,10 +368,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // ---------------------------------------------------------------------------
 // Skinny GEMM for decode (M <= 64 tokens): the weight is the streamed operand.
 // Swap-AB so the weight rows fill the M = 128 side of tcgen05.mma and the
-// tokens are N = 64; each CTA owns one 128-row weight tile and one slice of K
-// (split-K), so even N = 4096 keeps every SM streaming weights.  Output:
-// fp32 partial sums P[split][token][n] (row stride ldp), reduced by the
-// epilogue kernels.
+// tokens are N = 64.  Work items are (128-row weight tile, slice of K)
+// (split-K, so even N = 4096 keeps every SM streaming weights); a persistent
+// CTA per SM walks its items with the TMA ring and two TMEM accumulators
+// carried across items, so the epilogue of one item overlaps the next.
+// Output: fp32 partial sums P[split][token][n] (row stride ldp), reduced by
+// the epilogue kernels.
 // ---------------------------------------------------------------------------
 constexpr int SK_BN = 64, SK_STAGES = 6;
 constexpr int SK_A_BYTES = BM * BK * 2;     // weight tile 128 x 64
@@ -383,27 +385,31 @@ constexpr uint32_t SK_IDESC = idesc_bf16_f32(BM, SK_BN);
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmx, int M, int N,
                        int K, int splits, float* __restrict__ P, int64_t ldp, int* status) {
+  // persistent: CTA b takes items b, b + grid, ...; item = (split, weight tile)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sw_ = smem;
   uint8_t* sx = smem + SK_STAGES * SK_A_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SK_STAGES * SK_STAGE);
   uint64_t* empty = full + SK_STAGES;
-  uint64_t* tfull = empty + SK_STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
+  uint64_t* tfull = empty + SK_STAGES;  // 2 accumulators
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x, split = blockIdx.y;
+  const int tiles = (N + BM - 1) / BM, items = tiles * splits;
   const int kbs = K / BK;
-  const int kb0 = (int)((int64_t)kbs * split / splits), kb1 = (int)((int64_t)kbs * (split + 1) / splits);
   if (threadIdx.x == 0) {
     for (int s = 0; s < SK_STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(tfull, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
     fence_mbar_init();
   }
-  if (warp == 2) tmem_alloc(tmem_slot, SK_BN);
+  if (warp == 2) tmem_alloc(tmem_slot, 2 * SK_BN);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -413,51 +419,72 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tmap(&tmx);
     int stage = 0;
     uint32_t phase = 0;
-    for (int kb = kb0; kb < kb1; ++kb) {
-      if (!mbar_wait(&empty[stage], phase ^ 1, status, STATUS_WAIT_PRODUCER)) break;
-      mbar_expect_tx(&full[stage], SK_STAGE);
-      tma_load_2d(sw_ + stage * SK_A_BYTES, &tmw, &full[stage], kb * BK, tile * BM);
-      tma_load_2d(sx + stage * SK_B_BYTES, &tmx, &full[stage], kb * BK, 0);
-      if (++stage == SK_STAGES) { stage = 0; phase ^= 1; }
+    bool ok = true;
+    for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
+      const int split = it / tiles, tile = it % tiles;
+      const int kb0 = (int)((int64_t)kbs * split / splits), kb1 = (int)((int64_t)kbs * (split + 1) / splits);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, status, STATUS_WAIT_PRODUCER)) { ok = false; break; }
+        mbar_expect_tx(&full[stage], SK_STAGE);
+        tma_load_2d(sw_ + stage * SK_A_BYTES, &tmw, &full[stage], kb * BK, tile * BM);
+        tma_load_2d(sx + stage * SK_B_BYTES, &tmx, &full[stage], kb * BK, 0);
+        if (++stage == SK_STAGES) { stage = 0; phase ^= 1; }
+      }
     }
   } else if (warp == 1 && lane == 0) {
     int stage = 0;
     uint32_t phase = 0;
+    int local = 0;
     bool ok = true;
-    for (int kb = kb0; kb < kb1; ++kb) {
-      if (!mbar_wait(&full[stage], phase, status, STATUS_WAIT_MMA)) { ok = false; break; }
+    for (int it = blockIdx.x; it < items && ok; it += gridDim.x, ++local) {
+      const int split = it / tiles;
+      const int kb0 = (int)((int64_t)kbs * split / splits), kb1 = (int)((int64_t)kbs * (split + 1) / splits);
+      const int acc = local & 1;
+      if (!mbar_wait(&tempty[acc], ((local >> 1) & 1) ^ 1, status, STATUS_WAIT_MMA)) break;
       tc_fence_after();
-      const uint32_t a0 = smem_u32(sw_ + stage * SK_A_BYTES), b0 = smem_u32(sx + stage * SK_B_BYTES);
+      const uint32_t d = tmem + acc * SK_BN;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&full[stage], phase, status, STATUS_WAIT_MMA)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sw_ + stage * SK_A_BYTES), b0 = smem_u32(sx + stage * SK_B_BYTES);
 #pragma unroll
-      for (int k = 0; k < BK / 16; ++k)
-        tc_mma_f16(tmem, smem_desc_sw128(a0 + 32 * k, 1024), smem_desc_sw128(b0 + 32 * k, 1024), SK_IDESC,
-                   (kb > kb0 || k > 0) ? 1u : 0u);
-      tc_commit(&empty[stage]);
-      if (++stage == SK_STAGES) { stage = 0; phase ^= 1; }
+        for (int k = 0; k < BK / 16; ++k)
+          tc_mma_f16(d, smem_desc_sw128(a0 + 32 * k, 1024), smem_desc_sw128(b0 + 32 * k, 1024), SK_IDESC,
+                     (kb > kb0 || k > 0) ? 1u : 0u);
+        tc_commit(&empty[stage]);
+        if (++stage == SK_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (ok) tc_commit(&tfull[acc]);
     }
-    if (ok && kb1 > kb0) tc_commit(tfull);
   } else if (warp >= 4) {
     const int q = warp & 3;
-    const bool got = kb1 > kb0 && mbar_wait(tfull, 0, status, STATUS_WAIT_EPILOGUE);
-    if (__all_sync(0xffffffffu, got)) {
+    int local = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x, ++local) {
+      const int split = it / tiles, tile = it % tiles;
+      const int acc = local & 1;
+      const bool got = mbar_wait(&tfull[acc], (local >> 1) & 1, status, STATUS_WAIT_EPILOGUE);
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const int n = tile * BM + 32 * q + lane;
       float* dst = P + (int64_t)split * M * ldp + n;
 #pragma unroll 1
       for (int c = 0; c < SK_BN / 32; ++c) {
         float v[32];
-        ld_chunk(tmem + ((uint32_t)(32 * q) << 16) + 32 * c, v);
+        ld_chunk(tmem + acc * SK_BN + ((uint32_t)(32 * q) << 16) + 32 * c, v);
         if (n < N) {
           for (int j = 0; j < 32 && 32 * c + j < M; ++j) dst[(int64_t)(32 * c + j) * ldp] = v[j];
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, SK_BN);
+    tmem_dealloc(tmem, 2 * SK_BN);
   }
 }
 
@@ -522,9 +549,20 @@ cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, int M, int
 bool gemm_skinny_supported(int64_t M, int64_t N, int64_t K) { return M >= 1 && M <= SK_BN && K % BK == 0 && N > 0; }
 
 int gemm_skinny_splits(int64_t N, int64_t K) {
-  const int64_t tiles = (N + BM - 1) / BM, kbs = K / BK;
-  int64_t s = (2 * (int64_t)num_sms() + tiles - 1) / tiles;  // about two waves of CTAs
-  return (int)std::max<int64_t>(1, std::min<int64_t>({s, kbs, 32}));
+  // split-K count minimising the busiest CTA's work: items per CTA times
+  // (weight k-blocks per item + ~4 k-block equivalents of fp32 partials
+  // written and read back per item)
+  const int64_t tiles = (N + BM - 1) / BM, kbs = K / BK, sms = num_sms();
+  int best = 1;
+  double best_cost = (double)((tiles + sms - 1) / sms) * (double)kbs;  // one split writes no partials
+  for (int s = 2; s <= 16 && s <= kbs; ++s) {
+    const double cost = (double)((tiles * s + sms - 1) / sms) * ((double)kbs / s + 4.0);
+    if (cost < best_cost * 0.97) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
 }
 
 cudaError_t launch_gemm_skinny(const void* X, const void* W, int64_t M, int64_t N, int64_t K, int splits, float* P,
@@ -538,8 +576,9 @@ cudaError_t launch_gemm_skinny(const void* X, const void* W, int64_t M, int64_t 
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid((unsigned)((N + BM - 1) / BM), (unsigned)splits);
-  gemm_skinny_kernel<<<grid, THREADS, SK_SMEM, st>>>(mw, mx, (int)M, (int)N, (int)K, splits, P, ldp, status_ptr());
+  const int items = (int)((N + BM - 1) / BM) * splits;
+  gemm_skinny_kernel<<<std::min(items, num_sms()), THREADS, SK_SMEM, st>>>(mw, mx, (int)M, (int)N, (int)K, splits, P,
+                                                                         ldp, status_ptr());
   return cudaGetLastError();
 }
 

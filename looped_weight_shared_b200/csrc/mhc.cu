@@ -344,16 +344,39 @@ __global__ void __launch_bounds__(MHCB_WARPS * 32)
   }
 }
 
-// One-pass reader for H = 512 * NPL: one 128-thread CTA per token, each
-// thread keeps its NPL float4 of both streams in registers (loads issued
-// first), one lane forms the coefficients while those loads are in flight.
+// Coefficients of every token from its partial sums, one thread per token:
+// r, l = sum / r, H_pre, H_post and H_res = Sinkhorn(exp(l[4:8])).
+__global__ void __launch_bounds__(128)
+    mhc_coef_kernel(const float* __restrict__ part, int parts, int64_t T, int D, int iters, float eps,
+                    float* __restrict__ coef) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const float* pp = part + t * parts * 9;
+  float tot[9];
+#pragma unroll
+  for (int c = 0; c < 9; ++c) tot[c] = pp[c];
+  for (int q = 1; q < parts; ++q)
+#pragma unroll
+    for (int c = 0; c < 9; ++c) tot[c] += pp[q * 9 + c];
+  const float rinv = rsqrtf(tot[8] / D + eps);
+  float l[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) l[c] = tot[c] * rinv;
+  float P[4];
+  sinkhorn_fixed<2>(l + 4, P, iters);
+  float4* co = reinterpret_cast<float4*>(coef + t * 8);
+  co[0] = make_float4(sigmoidf_(l[0]), sigmoidf_(l[1]), 2.f * sigmoidf_(l[2]), 2.f * sigmoidf_(l[3]));
+  co[1] = make_float4(P[0], P[1], P[2], P[3]);
+}
+
+// One-pass reader for H = 512 * NPL (coefficients already formed): one
+// 128-thread CTA per token keeps its NPL float4 of both streams in registers,
+// so the stream rows are read once.
 template <typename T, int NPL>
 __global__ void __launch_bounds__(128)
-    mhc_read1_kernel(const float* __restrict__ s, int64_t Ttot, const float* __restrict__ part, int parts,
-                     const float* __restrict__ gain, int iters, float eps, float* __restrict__ coef,
-                     T* __restrict__ xh) {
+    mhc_read1_kernel(const float* __restrict__ s, int64_t Ttot, const float* __restrict__ coef,
+                     const float* __restrict__ gain, float eps, T* __restrict__ xh) {
   constexpr int H = 512 * NPL;
-  __shared__ float cf[2];
   __shared__ float red[4];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t t = blockIdx.x;
@@ -364,26 +387,7 @@ __global__ void __launch_bounds__(128)
   for (int i = 0; i < NPL; ++i) a[i] = __ldcs(s0 + tid + 128 * i);
 #pragma unroll
   for (int i = 0; i < NPL; ++i) b[i] = __ldcs(s1 + tid + 128 * i);
-  if (tid == 0) {
-    const float* pp = part + t * parts * 9;
-    float tot[9];
-    for (int c = 0; c < 9; ++c) tot[c] = pp[c];
-    for (int q = 1; q < parts; ++q)
-      for (int c = 0; c < 9; ++c) tot[c] += pp[q * 9 + c];
-    const float rinv = rsqrtf(tot[8] / (2 * H) + eps);
-    float l[8];
-    for (int c = 0; c < 8; ++c) l[c] = tot[c] * rinv;
-    float P[4];
-    sinkhorn_fixed<2>(l + 4, P, iters);
-    const float pre0 = sigmoidf_(l[0]), pre1 = sigmoidf_(l[1]);
-    cf[0] = pre0;
-    cf[1] = pre1;
-    float4* co = reinterpret_cast<float4*>(coef + t * 8);
-    co[0] = make_float4(pre0, pre1, 2.f * sigmoidf_(l[2]), 2.f * sigmoidf_(l[3]));
-    co[1] = make_float4(P[0], P[1], P[2], P[3]);
-  }
-  __syncthreads();
-  const float pre0 = cf[0], pre1 = cf[1];
+  const float pre0 = coef[t * 8], pre1 = coef[t * 8 + 1];
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
@@ -427,9 +431,10 @@ cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* g
   const int64_t per_cta = (int64_t)MHCA_WARPS * MHCA_TOK;
   dim3 ga((unsigned)((T + per_cta - 1) / per_cta), (unsigned)parts);
   mhc_partial_kernel<<<ga, MHCA_THREADS, smem, st>>>(s, T, H, gamma, phi, parts, part);
-  if (H == 4096) {  // the 9B width: one pass over the streams
-    if (bf) mhc_read1_kernel<bf16, 8><<<(unsigned)T, 128, 0, st>>>(s, T, part, parts, gain, iters, eps, coef, (bf16*)xh);
-    else mhc_read1_kernel<float, 8><<<(unsigned)T, 128, 0, st>>>(s, T, part, parts, gain, iters, eps, coef, (float*)xh);
+  if (H == 4096) {  // the 9B width: coefficients, then one pass over the streams
+    mhc_coef_kernel<<<(unsigned)((T + 127) / 128), 128, 0, st>>>(part, parts, T, 2 * H, iters, eps, coef);
+    if (bf) mhc_read1_kernel<bf16, 8><<<(unsigned)T, 128, 0, st>>>(s, T, coef, gain, eps, (bf16*)xh);
+    else mhc_read1_kernel<float, 8><<<(unsigned)T, 128, 0, st>>>(s, T, coef, gain, eps, (float*)xh);
     return cudaGetLastError();
   }
   const unsigned gb = (unsigned)((T + MHCB_WARPS - 1) / MHCB_WARPS);
