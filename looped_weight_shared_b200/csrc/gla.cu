@@ -8,9 +8,11 @@
 //   O   = ((Q K^T) * D) V + diag(exp b) Q S_prev,   D_ts = exp(b_t - b_s) [s <= t]
 //   S'  = exp(b_last) S_prev + K^T (diag(exp(b_last - b)) V).
 //
-// One CTA owns (sequence, head, 64-column slice of the value dimension) and
-// walks the chunks in order; its 128 x 64 fp32 state slice stays in MMA
-// accumulator registers for the whole sequence.  Q, K and the V slice of each
+// One CTA (8 warps) owns (sequence, head, 64-column slice of the value
+// dimension) and walks the chunks in order; its 128 x 64 fp32 state slice
+// stays in MMA accumulator registers for the whole sequence (16 rows per
+// warp).  Outputs: warp w computes rows 16 (w % 4) .. + 15 and value columns
+// 32 (w / 4) .. + 31 of the chunk.  Q, K and the V slice of each
 // chunk are staged by TMA (128-byte swizzle, double-buffered).  Products run
 // on bf16 mma.sync m16n8k16 with fp32 accumulation.  The three operands that
 // are not model activations - the state, the decayed scores (Q K^T) * D and
@@ -26,7 +28,7 @@ namespace loopk {
 
 namespace {
 
-constexpr int C = 64, DK = 128, DV = 64, WARPS = 4, THREADS = WARPS * 32;
+constexpr int C = 64, DK = 128, DV = 64, WARPS = 8, THREADS = WARPS * 32;
 constexpr int QK_BYTES = C * DK * 2;            // Q or K tile: two boxes [64][64]
 constexpr int V_BYTES = C * DV * 2;             // V slice: one box [64][64]
 constexpr int STAGE_BYTES = 2 * QK_BYTES + V_BYTES;
@@ -81,21 +83,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (nch > 1) issue(1);
   }
 
-  // state slice: warp w owns rows 32w .. 32w + 31 (two m16 tiles) x 64 columns
-  float acc[2][8][4];
+  // state slice: warp w owns rows 16w .. 16w + 15 (one m16 tile) x 64 columns
+  float acc[8][4];
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int r = warp * 32 + mt * 16 + g, c = nt * 8 + 2 * t;
-      acc[mt][nt][0] = st[(int64_t)r * 128 + c];
-      acc[mt][nt][1] = st[(int64_t)r * 128 + c + 1];
-      acc[mt][nt][2] = st[(int64_t)(r + 8) * 128 + c];
-      acc[mt][nt][3] = st[(int64_t)(r + 8) * 128 + c + 1];
-    }
+  for (int nt = 0; nt < 8; ++nt) {
+    const int r = warp * 16 + g, c = nt * 8 + 2 * t;
+    acc[nt][0] = st[(int64_t)r * 128 + c];
+    acc[nt][1] = st[(int64_t)r * 128 + c + 1];
+    acc[nt][2] = st[(int64_t)(r + 8) * 128 + c];
+    acc[nt][3] = st[(int64_t)(r + 8) * 128 + c + 1];
+  }
 
   const uint32_t shi_u = smem_u32(shi), slo_u = smem_u32(slo), vhat_u = smem_u32(vhat),
                  vlo_u = smem_u32(vhat_lo);
+  const int rg = warp & 3, ch = warp >> 2;  // output phase: rows 16 rg .., value columns 32 ch ..
   for (int c = 0; c < nch; ++c) {
     const int c0 = c * C;
     const int valid = min(C, S - c0);
@@ -118,28 +119,26 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     // current state as bf16 hi + lo, row-major [dk][64] with the 128-byte swizzle
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = warp * 32 + mt * 16 + g + 8 * hf;
-          const float x0 = acc[mt][nt][2 * hf], x1 = acc[mt][nt][2 * hf + 1];
-          const __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
-          const float2 hf2 = __bfloat1622float2(hi);
-          const __nv_bfloat162 lo = __floats2bfloat162_rn(x0 - hf2.x, x1 - hf2.y);
-          const uint32_t off = (uint32_t)(r * 128 + ((nt ^ (r & 7)) << 4) + 4 * t);
-          *reinterpret_cast<__nv_bfloat162*>(shi + off) = hi;
-          *reinterpret_cast<__nv_bfloat162*>(slo + off) = lo;
-        }
+      for (int hf = 0; hf < 2; ++hf) {
+        const int r = warp * 16 + g + 8 * hf;
+        const float x0 = acc[nt][2 * hf], x1 = acc[nt][2 * hf + 1];
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
+        const float2 hf2 = __bfloat1622float2(hi);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(x0 - hf2.x, x1 - hf2.y);
+        const uint32_t off = (uint32_t)(r * 128 + ((nt ^ (r & 7)) << 4) + 4 * t);
+        *reinterpret_cast<__nv_bfloat162*>(shi + off) = hi;
+        *reinterpret_cast<__nv_bfloat162*>(slo + off) = lo;
+      }
     __syncthreads();
     const float b_last = bv[C - 1];
     uint8_t* sg = stage0 + (c & 1) * STAGE_BYTES;
     const uint32_t q_u = smem_u32(sg), k_u = q_u + QK_BYTES, v_u = q_u + 2 * QK_BYTES;
-    // V-hat = diag(exp(b_last - b)) V, zero past the end of the sequence
+    // V-hat = diag(exp(b_last - b)) V as hi + lo, zero past the end of the sequence
     for (int ci = tid; ci < C * 8; ci += THREADS) {
-      const int r = ci >> 3, ch = ci & 7;
-      const uint32_t off = (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
+      const int r = ci >> 3, chk = ci & 7;
+      const uint32_t off = (uint32_t)(r * 128 + ((chk ^ (r & 7)) << 4));
       const float f = r < valid ? __expf(b_last - bv[r]) : 0.f;
       uint4 u = *reinterpret_cast<const uint4*>(sg + 2 * QK_BYTES + off);
       uint4 w;
@@ -158,12 +157,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncthreads();
 
-    // ---- outputs of rows 16w .. 16w + 15 of the chunk ----
+    // ---- outputs: rows 16 rg .. 16 rg + 15, value columns 32 ch .. 32 ch + 31 ----
     {
       uint32_t qf[8][4];
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        ldsm_x4(q_u + sw(warp * 16 + (mi & 1) * 8 + ri, kk * 2 + (mi >> 1), C), qf[kk][0], qf[kk][1], qf[kk][2],
+        ldsm_x4(q_u + sw(rg * 16 + (mi & 1) * 8 + ri, kk * 2 + (mi >> 1), C), qf[kk][0], qf[kk][1], qf[kk][2],
                 qf[kk][3]);
       float a[8][4];
 #pragma unroll
@@ -177,7 +176,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           mma_bf16(a[nt], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
           mma_bf16(a[nt + 1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
         }
-      const int tq0 = warp * 16 + g, tq1 = tq0 + 8;
+      const int tq0 = rg * 16 + g, tq1 = tq0 + 8;
       const float bt0 = bv[tq0], bt1 = bv[tq1];
       uint32_t pa[8][2], pl[8][2];  // (Q K^T) * D as bf16 hi + lo
 #pragma unroll
@@ -185,10 +184,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         float d[4];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int s = nt * 8 + 2 * t + e;
-          const float bs = bv[s];
-          d[e] = (s <= tq0 && s < valid) ? __expf(bt0 - bs) : 0.f;
-          d[2 + e] = (s <= tq1 && s < valid) ? __expf(bt1 - bs) : 0.f;
+          const int sk = nt * 8 + 2 * t + e;
+          const float bs = bv[sk];
+          d[e] = (sk <= tq0 && sk < valid) ? __expf(bt0 - bs) : 0.f;
+          d[2 + e] = (sk <= tq1 && sk < valid) ? __expf(bt1 - bs) : 0.f;
         }
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
@@ -201,15 +200,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // inter-chunk first: o = exp(b_t) Q S_prev (S as hi + lo), then the
       // intra-chunk (A * D) V accumulates onto it
-      float o[8][4];
+      float o[4][4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+      for (int i = 0; i < 4; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
 #pragma unroll
-        for (int nt = 0; nt < 8; nt += 2) {
+        for (int nt = 0; nt < 4; nt += 2) {
           uint32_t b0, b1, b2, b3;
-          const uint32_t off = sw(kk * 16 + (mi & 1) * 8 + ri, nt + (mi >> 1), DK);
+          const uint32_t off = sw(kk * 16 + (mi & 1) * 8 + ri, ch * 4 + nt + (mi >> 1), DK);
           ldsm_x4_t(shi_u + off, b0, b1, b2, b3);
           mma_bf16(o[nt], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
           mma_bf16(o[nt + 1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
@@ -219,7 +218,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       const float e0 = __expf(bt0), e1 = __expf(bt1);
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int nt = 0; nt < 4; ++nt) {
         o[nt][0] *= e0;
         o[nt][1] *= e0;
         o[nt][2] *= e1;
@@ -228,58 +227,45 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-        for (int nt = 0; nt < 8; nt += 2) {
+        for (int nt = 0; nt < 4; nt += 2) {
           uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(v_u + sw(kk * 16 + (mi & 1) * 8 + ri, nt + (mi >> 1), C), b0, b1, b2, b3);
+          ldsm_x4_t(v_u + sw(kk * 16 + (mi & 1) * 8 + ri, ch * 4 + nt + (mi >> 1), C), b0, b1, b2, b3);
           mma_bf16(o[nt], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b0, b1);
           mma_bf16(o[nt + 1], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b2, b3);
           mma_bf16(o[nt], pl[2 * kk][0], pl[2 * kk][1], pl[2 * kk + 1][0], pl[2 * kk + 1][1], b0, b1);
           mma_bf16(o[nt + 1], pl[2 * kk][0], pl[2 * kk][1], pl[2 * kk + 1][0], pl[2 * kk + 1][1], b2, b3);
         }
       const int64_t ld = (int64_t)nh * 128;
-      bf16* r0p = out + ((int64_t)b * S + c0 + tq0) * ld + h * 128 + slice * DV;
-      bf16* r1p = out + ((int64_t)b * S + c0 + tq1) * ld + h * 128 + slice * DV;
+      bf16* r0p = out + ((int64_t)b * S + c0 + tq0) * ld + h * 128 + slice * DV + ch * 32;
+      bf16* r1p = out + ((int64_t)b * S + c0 + tq1) * ld + h * 128 + slice * DV + ch * 32;
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int nt = 0; nt < 4; ++nt) {
         const int col = nt * 8 + 2 * t;
         if (tq0 < valid) *reinterpret_cast<uint32_t*>(r0p + col) = pack_bf16x2(o[nt][0], o[nt][1]);
         if (tq1 < valid) *reinterpret_cast<uint32_t*>(r1p + col) = pack_bf16x2(o[nt][2], o[nt][3]);
       }
     }
-    // ---- state update: S = exp(b_last) S + K^T V-hat ----
+    // ---- state update: S = exp(b_last) S + K^T V-hat (rows 16 warp ..) ----
     {
       const float dl = __expf(b_last);
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
+      for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[mt][nt][e] *= dl;
+        for (int e = 0; e < 4; ++e) acc[nt][e] *= dl;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        uint32_t af[2][4];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          const int dk0 = warp * 32 + mt * 16;
-          ldsm_x4_t(k_u + sw(kk * 16 + (mi >> 1) * 8 + ri, dk0 / 8 + (mi & 1), C), af[mt][0], af[mt][1], af[mt][2],
-                    af[mt][3]);
-        }
+        uint32_t af[4];
+        ldsm_x4_t(k_u + sw(kk * 16 + (mi >> 1) * 8 + ri, 2 * warp + (mi & 1), C), af[0], af[1], af[2], af[3]);
 #pragma unroll
         for (int nt = 0; nt < 8; nt += 2) {
           uint32_t b0, b1, b2, b3;
           const uint32_t off = sw(kk * 16 + (mi & 1) * 8 + ri, nt + (mi >> 1), C);
           ldsm_x4_t(vhat_u + off, b0, b1, b2, b3);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            mma_bf16(acc[mt][nt], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b0, b1);
-            mma_bf16(acc[mt][nt + 1], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b2, b3);
-          }
+          mma_bf16(acc[nt], af[0], af[1], af[2], af[3], b0, b1);
+          mma_bf16(acc[nt + 1], af[0], af[1], af[2], af[3], b2, b3);
           ldsm_x4_t(vlo_u + off, b0, b1, b2, b3);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            mma_bf16(acc[mt][nt], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b0, b1);
-            mma_bf16(acc[mt][nt + 1], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b2, b3);
-          }
+          mma_bf16(acc[nt], af[0], af[1], af[2], af[3], b0, b1);
+          mma_bf16(acc[nt + 1], af[0], af[1], af[2], af[3], b2, b3);
         }
       }
     }
@@ -287,17 +273,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (tid == 0 && c + 2 < nch) issue(c + 2);
   }
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int r = warp * 32 + mt * 16 + g, c = nt * 8 + 2 * t;
-      st[(int64_t)r * 128 + c] = acc[mt][nt][0];
-      st[(int64_t)r * 128 + c + 1] = acc[mt][nt][1];
-      st[(int64_t)(r + 8) * 128 + c] = acc[mt][nt][2];
-      st[(int64_t)(r + 8) * 128 + c + 1] = acc[mt][nt][3];
-    }
+  for (int nt = 0; nt < 8; ++nt) {
+    const int r = warp * 16 + g, c = nt * 8 + 2 * t;
+    st[(int64_t)r * 128 + c] = acc[nt][0];
+    st[(int64_t)r * 128 + c + 1] = acc[nt][1];
+    st[(int64_t)(r + 8) * 128 + c] = acc[nt][2];
+    st[(int64_t)(r + 8) * 128 + c + 1] = acc[nt][3];
+  }
 }
-
 
 // ---------------------------------------------------------------------------
 // One decode step of gated linear attention (d = 128): S = g S + k v^T,

@@ -419,7 +419,7 @@ size_t mhc_partial_smem(int H) { return (size_t)9 * H * sizeof(float); }
 
 cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf,
-                                float* part, cudaStream_t st, int parts) {
+                                float* part, cudaStream_t st, int parts, bool fused_read) {
   if (T == 0) return cudaSuccess;
   if (H % 4 != 0 || mhc_partial_smem(H) > 220 * 1024) return cudaErrorInvalidValue;
   if (parts < 2 || parts % 2 != 0 || (2 * H) % (4 * parts) != 0 || H % (2 * H / parts) != 0)
@@ -431,7 +431,7 @@ cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* g
   const int64_t per_cta = (int64_t)MHCA_WARPS * MHCA_TOK;
   dim3 ga((unsigned)((T + per_cta - 1) / per_cta), (unsigned)parts);
   mhc_partial_kernel<<<ga, MHCA_THREADS, smem, st>>>(s, T, H, gamma, phi, parts, part);
-  if (H == 4096) {  // the 9B width: coefficients, then one pass over the streams
+  if (H == 4096 && !fused_read) {  // the 9B width: coefficients, then one pass over the streams
     mhc_coef_kernel<<<(unsigned)((T + 127) / 128), 128, 0, st>>>(part, parts, T, 2 * H, iters, eps, coef);
     if (bf) mhc_read1_kernel<bf16, 8><<<(unsigned)T, 128, 0, st>>>(s, T, coef, gain, eps, (bf16*)xh);
     else mhc_read1_kernel<float, 8><<<(unsigned)T, 128, 0, st>>>(s, T, coef, gain, eps, (float*)xh);

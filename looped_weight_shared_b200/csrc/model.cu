@@ -522,10 +522,12 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
         // decode (few tokens): cut Phi into 16 parts so the partial kernel spreads over the SMs;
         // a prefill always uses 2, so each row's arithmetic is the same at any length
         const int parts = (m.decoding && H % 32 == 0 && T * 16 * 9 <= w.mhc_part_floats) ? 16 : 2;
-        LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), H == 4096 ? 3 : 2, st, [&] {
-          return launch_mhc_prologue(s_buf, T, (int)H, site.gamma, site.phi, gain, c.sinkhorn_iters, c.norm_eps,
-                                     w.coef, w.xh, bf, w.mhc_part, st, parts);
-        }));
+        // decode uses the reader that forms the coefficients itself (one launch less per site)
+        LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), (H == 4096 && !m.decoding) ? 3 : 2, st,
+                      [&] {
+                        return launch_mhc_prologue(s_buf, T, (int)H, site.gamma, site.phi, gain, c.sinkhorn_iters,
+                                                   c.norm_eps, w.coef, w.xh, bf, w.mhc_part, st, parts, m.decoding);
+                      }));
       } else {
         LOOP_CU(timed(m, LOOP_K_NORM, (double)T * H * (4 + es), 1, st,
                       [&] { return launch_rmsnorm(w.h, T, (int)H, 1, 0, gain, c.norm_eps, w.xh, bf, st); }));

@@ -132,11 +132,14 @@ cudaError_t launch_embed(const int32_t* tok, const void* E, bool bf16, int64_t T
                          cudaStream_t st);
 cudaError_t launch_rmsnorm(const float* x, int64_t rows, int H, int64_t row_step, int64_t row_off,
                            const float* gain, float eps, void* y, bool bf16, cudaStream_t st);
-// two kernels; `part` is scratch of 9 x parts floats per token (parts even,
-// dividing the stream width into equal float4 runs; 2 by default)
+// two or three kernels; `part` is scratch of 9 x parts floats per token
+// (parts even, dividing the stream width into equal float4 runs; 2 by
+// default).  fused_read selects the reader that forms the coefficients
+// itself (fewer launches for a few tokens) at every width; otherwise hidden
+// 4096 uses a coefficient kernel and a one-pass reader.
 cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf16,
-                                float* part, cudaStream_t st, int parts = 2);
+                                float* part, cudaStream_t st, int parts = 2, bool fused_read = false);
 size_t mhc_partial_smem(int H);
 cudaError_t launch_expand(const float* h, float* s, int64_t n, cudaStream_t st);
 cudaError_t launch_collapse(const float* s, float* h, int64_t n, cudaStream_t st);
