@@ -29,6 +29,15 @@ import seeded  # noqa: E402
 from seeded import workloads as W  # noqa: E402
 
 DEFAULT_WORKLOAD = "loop9b_prefill_b4_s8192"
+
+# DRAM read + write per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum):
+# - tcgen05 GEMM: mean over the 675 GEMM launches of three 9B prefill steps
+#   (a single-pass ncu launch list of `bench.py --steps 1 --warmup 1`)
+# - decode attention: 1.085 GB per launch on the probe_decode_b64_ctx4096
+#   workload (64 x 4096 keys), scaled by keys to 32,787
+# Set to None when the kernel changes after the capture.
+GEMM_TRAFFIC_PER_LAUNCH = 3.97e9
+DECODE_ATTN_TRAFFIC_PER_LAUNCH = 1.085e9 * 32787 / 4097
 DATA = "synthetic: seeded SplitMix64 token ids, random-init N(0, 0.02) bf16 weights of the 9B shape"
 
 
@@ -426,7 +435,8 @@ def main():
     peak = pk["bf16_tflops_sustained"]
     roof = {"bound": "tensor", "kernel": "tcgen05 projection GEMM (all launches in the timed steps)",
             "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak if peak else None,
-            "peak_kind": f"{pk_kind} sustained bf16", "traffic": None}
+            "peak_kind": f"{pk_kind} sustained bf16", "traffic": GEMM_TRAFFIC_PER_LAUNCH,
+            "traffic_note": "mean DRAM bytes per GEMM launch (ncu); achieved is over all GEMM launches of the steps"}
     line = {"metric": metric, "value": r["value"], "unit": unit, "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": DATA, "config": config, "clocks": r["clocks"],
@@ -448,7 +458,9 @@ def main():
             "step_roofline": {"bound": "hbm", "achieved": step_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                               "frac": step_gbs / pk["hbm_gbs"], "peak_kind": f"{pk_kind} copy bandwidth"},
             "roofline": {"bound": "hbm", "kernel": "decode attention (KV-cache read)", "achieved": kv_gbs,
-                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": kv_gbs / pk["hbm_gbs"], "traffic": None},
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": kv_gbs / pk["hbm_gbs"],
+                         "traffic": DECODE_ATTN_TRAFFIC_PER_LAUNCH,
+                         "traffic_note": "per launch, scaled by context from a 4096-key capture"},
             "kernel_ms_per_step": {k: round(v["ms_per_step"], 3) for k, v in d["classes"].items()},
             "kernel_split_note": "per-class times come from a second run of the same steps with CUDA events around "
                                  "every launch (ms_per_step_with_launch_events); the headline ms_per_step has none",

@@ -224,11 +224,20 @@ LOOP_API int32_t loop_timing_read(loop_model* m, int32_t cls, double* total_ms, 
 /* Number of kernels this model has launched since it was created. */
 LOOP_API int64_t loop_launch_count(const loop_model* m);
 
-/* Sticky device status word: 0, or the bits of waits that timed out in a
- * kernel (the kernel then returned early).  Reading it synchronises the
+/* Sticky device status word: 0, or bits for what went wrong in a kernel: 1
+ * TMA producer wait, 2 MMA-issuer wait, 4 epilogue / consumer wait, 8 other
+ * wait timed out (the kernel then returned early); 16 a token id outside
+ * [0, vocab) was embedded as zeros; 32 the self-test timeout fired.  Reading it synchronises the
  * device.  loop_clear_device_status() resets it. */
 LOOP_API int32_t loop_device_status(void);
 LOOP_API void loop_clear_device_status(void);
+
+/* Failure-detection self-test: one kernel waits on an mbarrier phase that
+ * never completes, with a limit of timeout_ms; the wait gives up, records bit
+ * 32 (self-test) in the status word and the kernel returns normally, so the
+ * context stays usable.  Synchronises; returns the status word (the caller
+ * clears it with loop_clear_device_status) or a negative LOOP_E* code. */
+LOOP_API int32_t loop_selftest_timeout(int32_t timeout_ms);
 
 /* Text of the last failed call on this thread ("" if none). */
 LOOP_API const char* loop_last_error(void);

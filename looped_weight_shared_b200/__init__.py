@@ -26,7 +26,7 @@ API = ("loop_num_exec", "loop_schedule", "loop_num_weights", "loop_model_create"
        "loop_decode_step", "mhc_sinkhorn", "loop_model_destroy", "loop_seq_len", "loop_cache_read",
        "loop_weight_read", "loop_device_status", "loop_clear_device_status", "loop_last_error",
        "loop_gemm_bf16", "loop_set_timing", "loop_timing_read", "loop_launch_count", "mhc_prologue",
-       "mhc_prologue_noalloc")
+       "mhc_prologue_noalloc", "loop_selftest_timeout")
 
 
 class loop_config(C.Structure):
@@ -82,6 +82,7 @@ def lib():
             "loop_launch_count": (C.c_int64, [vp]),
             "mhc_prologue": (i32, [vp, C.c_int64, i32, vp, vp, vp, i32, C.c_float, vp, vp, i32, vp, vp]),
             "mhc_prologue_noalloc": (i32, [vp, C.c_int64, i32, vp, vp, vp, i32, C.c_float, vp, vp, i32, vp]),
+            "loop_selftest_timeout": (i32, [i32]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -190,6 +191,14 @@ def loop_device_status() -> int:
 
 def loop_clear_device_status() -> None:
     lib().loop_clear_device_status()
+
+
+STATUS_WAIT_PRODUCER, STATUS_WAIT_MMA, STATUS_WAIT_EPILOGUE, STATUS_WAIT_OTHER = 1, 2, 4, 8
+STATUS_BAD_TOKEN, STATUS_SELFTEST = 16, 32
+
+
+def loop_selftest_timeout(timeout_ms: int = 50) -> int:
+    return _check("loop_selftest_timeout", lib().loop_selftest_timeout(timeout_ms))
 
 
 def loop_gemm_bf16(A, W, C_out, use_tensor_cores: bool = True, stream=None) -> None:

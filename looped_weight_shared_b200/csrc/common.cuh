@@ -23,6 +23,7 @@ enum : int {
   STATUS_WAIT_EPILOGUE = 4,
   STATUS_WAIT_OTHER = 8,
   STATUS_BAD_TOKEN = 16,
+  STATUS_SELFTEST = 32,
 };
 // `st` is the library's status word (see status_ptr()); NULL disables flagging.
 LOOP_DEV void flag_status(int* st, int bits) {
@@ -107,14 +108,14 @@ LOOP_DEV uint64_t globaltimer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Wait for phase `parity` of `bar`; gives up after ~2 s, ORs `who` into the
-// status word and returns false.
-LOOP_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* st, int who) {
+// Wait for phase `parity` of `bar`; gives up after `limit_ns` (2 s by
+// default), ORs `who` into the status word and returns false.
+LOOP_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* st, int who, uint64_t limit_ns = 2000000000ull) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 255u && globaltimer_ns() - t0 > 2000000000ull) {
+    if ((it & 255u) == 255u && globaltimer_ns() - t0 > limit_ns) {
       flag_status(st, who);
       return false;
     }

@@ -562,3 +562,21 @@ void status_clear() {
   cudaMemcpyToSymbol(g_status, &z, sizeof(int));
 }
 }  // namespace loopk
+
+namespace loopk {
+// A wait that nothing will end: one thread waits on a fresh mbarrier whose
+// phase never completes, with a short limit, so the timeout path runs.
+__global__ void selftest_timeout_kernel(uint64_t limit_ns, int* status, int* result) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) *result = mbar_wait(&bar, 0, status, STATUS_SELFTEST, limit_ns) ? 1 : 0;
+}
+cudaError_t launch_selftest_timeout(uint64_t limit_ns, int* result, cudaStream_t st) {
+  selftest_timeout_kernel<<<1, 32, 0, st>>>(limit_ns, status_ptr(), result);
+  return cudaGetLastError();
+}
+}  // namespace loopk

@@ -804,6 +804,22 @@ int32_t loop_device_status(void) {
 
 void loop_clear_device_status(void) { status_clear(); }
 
+int32_t loop_selftest_timeout(int32_t timeout_ms) {
+  if (timeout_ms < 1 || timeout_ms > 10000) return fail(LOOP_EINVAL, "timeout_ms in [1, 10000]");
+  int* d = nullptr;
+  if (cudaMalloc(&d, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LOOP_ENOMEM, "cudaMalloc failed");
+  }
+  int r = -1;
+  cudaError_t e = launch_selftest_timeout((uint64_t)timeout_ms * 1000000ull, d, 0);
+  if (e == cudaSuccess) e = cudaMemcpy(&r, d, sizeof(int), cudaMemcpyDeviceToHost);
+  cudaFree(d);
+  if (e != cudaSuccess) return fail(LOOP_ECUDA, cudaGetErrorString(e));
+  if (r != 0) return fail(LOOP_ECUDA, "the self-test wait completed, which nothing should cause");
+  return loop_device_status();
+}
+
 const char* loop_last_error(void) { return g_last_error.c_str(); }
 
 int32_t loop_gemm_bf16(const void* d_A, const void* d_W, int64_t M, int64_t N, int64_t K, float* d_C, int64_t ldc,

@@ -159,6 +159,7 @@ cudaError_t launch_rope_table(float2* tab, int64_t ctx, int hd, double base, cud
 cudaError_t launch_cache_to_f32(const void* src, bool bf16, int B, int nkv, int64_t ctx, int len, int hd,
                                 float* dst, cudaStream_t st);
 cudaError_t launch_advance(int32_t* seq_len, int B, cudaStream_t st);
+cudaError_t launch_selftest_timeout(uint64_t limit_ns, int* result, cudaStream_t st);
 cudaError_t launch_set_len(int32_t* seq_len, int B, int S, cudaStream_t st);
 cudaError_t launch_weight_to_f32(const void* src, bool bf16, int64_t rows, int64_t cols, int64_t src_row0,
                                  float* dst, cudaStream_t st);

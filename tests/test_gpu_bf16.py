@@ -79,7 +79,7 @@ def test_group9b_bf16_matches_oracle(S):
 MID = dict(hidden=512, ffn=512, vocab=2048, n_q=4, n_kv=2, head_dim=128, n_lin=4, lin_dim=128, dtype=1)
 
 
-@pytest.mark.parametrize("B,S", [(2, 700), (1, 64), (3, 129)])
+@pytest.mark.parametrize("B,S", [(2, 700), (1, 64), (3, 129), (2, 1)])
 def test_mid_bf16_all_positions(B, S):
     """head_dim 128 (the flash-attention and fused-epilogue shapes) with a
     narrow model so the oracle stays fast: several ragged query blocks."""
