@@ -415,6 +415,115 @@ __global__ void __launch_bounds__(128)
   }
 }
 
+// Whole mHC read site for a few tokens (decode): one 256-thread CTA per token
+// streams the token's two stream rows once (each thread keeps NK float4 of
+// both streams), dots them with gamma * Phi read from L2, reduces the 9 sums
+// over the CTA, forms the coefficients in one thread (Sinkhorn included), and
+// normalises x = H_pre s from registers.  One launch, no scratch.
+template <typename T, int NK>
+__global__ void __launch_bounds__(256)
+    mhc_token_kernel(const float* __restrict__ s, int64_t Ttot, const float* __restrict__ gamma,
+                     const float* __restrict__ phi, const float* __restrict__ gain, int iters, float eps,
+                     float* __restrict__ coef, T* __restrict__ xh) {
+  constexpr int H = 1024 * NK, H4 = H / 4, D = 2 * H;
+  __shared__ float red[8][9];
+  __shared__ float cf[2];
+  __shared__ float red2[8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t = blockIdx.x;
+  const float4* s0 = reinterpret_cast<const float4*>(s + t * H);
+  const float4* s1 = reinterpret_cast<const float4*>(s + (Ttot + t) * H);
+  float4 a[NK], b[NK];
+#pragma unroll
+  for (int k = 0; k < NK; ++k) a[k] = s0[tid + 256 * k];
+#pragma unroll
+  for (int k = 0; k < NK; ++k) b[k] = s1[tid + 256 * k];
+  float acc[9];
+#pragma unroll
+  for (int c = 0; c < 9; ++c) acc[c] = 0.f;
+  const float4* g4 = reinterpret_cast<const float4*>(gamma);
+#pragma unroll
+  for (int k = 0; k < 2 * NK; ++k) {
+    const float4 v = k < NK ? a[k] : b[k - NK];
+    const int f = (k < NK ? 0 : H4) + tid + 256 * (k % NK);
+    const float4 g = g4[f];
+    const float4 w = make_float4(v.x * g.x, v.y * g.y, v.z * g.z, v.w * g.w);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 p = reinterpret_cast<const float4*>(phi + (int64_t)c * D)[f];
+      acc[c] += w.x * p.x + w.y * p.y + w.z * p.z + w.w * p.w;
+    }
+    acc[8] += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+#pragma unroll
+  for (int c = 0; c < 9; ++c) {
+    const float r = warp_sum(acc[c]);
+    if (lane == 0) red[warp][c] = r;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float tot[9];
+    for (int c = 0; c < 9; ++c) {
+      float x = 0.f;
+      for (int w = 0; w < 8; ++w) x += red[w][c];
+      tot[c] = x;
+    }
+    const float rinv = rsqrtf(tot[8] / D + eps);
+    float l[8];
+    for (int c = 0; c < 8; ++c) l[c] = tot[c] * rinv;
+    float P[4];
+    sinkhorn_fixed<2>(l + 4, P, iters);
+    const float pre0 = sigmoidf_(l[0]), pre1 = sigmoidf_(l[1]);
+    cf[0] = pre0;
+    cf[1] = pre1;
+    float4* co = reinterpret_cast<float4*>(coef + t * 8);
+    co[0] = make_float4(pre0, pre1, 2.f * sigmoidf_(l[2]), 2.f * sigmoidf_(l[3]));
+    co[1] = make_float4(P[0], P[1], P[2], P[3]);
+  }
+  __syncthreads();
+  const float pre0 = cf[0], pre1 = cf[1];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < NK; ++k) {
+    a[k] = make_float4(pre0 * a[k].x + pre1 * b[k].x, pre0 * a[k].y + pre1 * b[k].y, pre0 * a[k].z + pre1 * b[k].z,
+                       pre0 * a[k].w + pre1 * b[k].w);
+    ss += a[k].x * a[k].x + a[k].y * a[k].y + a[k].z * a[k].z + a[k].w * a[k].w;
+  }
+  ss = warp_sum(ss);
+  if (lane == 0) red2[warp] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red2[w];
+  const float nrm = rsqrtf(tot / H + eps);
+  const float4* gn = reinterpret_cast<const float4*>(gain);
+#pragma unroll
+  for (int k = 0; k < NK; ++k) {
+    const int f = tid + 256 * k;
+    const float4 g = gn[f];
+    const float x0 = a[k].x * nrm * g.x, x1 = a[k].y * nrm * g.y, x2 = a[k].z * nrm * g.z, x3 = a[k].w * nrm * g.w;
+    if constexpr (sizeof(T) == 2) {
+      uint2 u;
+      u.x = pack_bf16x2(x0, x1);
+      u.y = pack_bf16x2(x2, x3);
+      reinterpret_cast<uint2*>(xh + t * H)[f] = u;
+    } else {
+      reinterpret_cast<float4*>(xh + t * H)[f] = make_float4(x0, x1, x2, x3);
+    }
+  }
+}
+
+bool mhc_token_supported(int H) { return H == 4096; }
+
+cudaError_t launch_mhc_token(const float* s, int64_t T, int H, const float* gamma, const float* phi,
+                             const float* gain, int iters, float eps, float* coef, void* xh, bool bf, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (H != 4096) return cudaErrorInvalidValue;
+  if (bf) mhc_token_kernel<bf16, 4><<<(unsigned)T, 256, 0, st>>>(s, T, gamma, phi, gain, iters, eps, coef, (bf16*)xh);
+  else mhc_token_kernel<float, 4><<<(unsigned)T, 256, 0, st>>>(s, T, gamma, phi, gain, iters, eps, coef, (float*)xh);
+  return cudaGetLastError();
+}
+
 size_t mhc_partial_smem(int H) { return (size_t)9 * H * sizeof(float); }
 
 cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,

@@ -519,15 +519,23 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
       const float* gain = sub == 0 ? L.attn_gain : L.ffn_gain;
       if (in_block) {
         const SiteW& site = m.sites[2 * (phys - c.n_prelude) + sub];
-        // decode (few tokens): cut Phi into 16 parts so the partial kernel spreads over the SMs;
-        // a prefill always uses 2, so each row's arithmetic is the same at any length
-        const int parts = (m.decoding && H % 32 == 0 && T * 16 * 9 <= w.mhc_part_floats) ? 16 : 2;
-        // decode uses the reader that forms the coefficients itself (one launch less per site)
-        LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), (H == 4096 && !m.decoding) ? 3 : 2, st,
-                      [&] {
-                        return launch_mhc_prologue(s_buf, T, (int)H, site.gamma, site.phi, gain, c.sinkhorn_iters,
-                                                   c.norm_eps, w.coef, w.xh, bf, w.mhc_part, st, parts, m.decoding);
-                      }));
+        if (m.decoding && mhc_token_supported((int)H)) {  // decode: one CTA per token, one launch
+          LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), 1, st, [&] {
+            return launch_mhc_token(s_buf, T, (int)H, site.gamma, site.phi, gain, c.sinkhorn_iters, c.norm_eps,
+                                    w.coef, w.xh, bf, st);
+          }));
+        } else {
+          // decode at other widths: cut Phi into 16 parts so the partial kernel spreads over the
+          // SMs and use the reader that forms the coefficients itself; a prefill always uses 2
+          // parts and (at hidden 4096) the coefficient kernel, so each row's arithmetic is the
+          // same at any length
+          const int parts = (m.decoding && H % 32 == 0 && T * 16 * 9 <= w.mhc_part_floats) ? 16 : 2;
+          LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), (H == 4096 && !m.decoding) ? 3 : 2,
+                        st, [&] {
+                          return launch_mhc_prologue(s_buf, T, (int)H, site.gamma, site.phi, gain, c.sinkhorn_iters,
+                                                     c.norm_eps, w.coef, w.xh, bf, w.mhc_part, st, parts, m.decoding);
+                        }));
+        }
       } else {
         LOOP_CU(timed(m, LOOP_K_NORM, (double)T * H * (4 + es), 1, st,
                       [&] { return launch_rmsnorm(w.h, T, (int)H, 1, 0, gain, c.norm_eps, w.xh, bf, st); }));

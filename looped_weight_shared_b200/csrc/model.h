@@ -141,6 +141,10 @@ cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* g
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf16,
                                 float* part, cudaStream_t st, int parts = 2, bool fused_read = false);
 size_t mhc_partial_smem(int H);
+// one launch per site for a few tokens (decode), hidden 4096
+bool mhc_token_supported(int H);
+cudaError_t launch_mhc_token(const float* s, int64_t T, int H, const float* gamma, const float* phi,
+                             const float* gain, int iters, float eps, float* coef, void* xh, bool bf16, cudaStream_t st);
 cudaError_t launch_expand(const float* h, float* s, int64_t n, cudaStream_t st);
 cudaError_t launch_collapse(const float* s, float* h, int64_t n, cudaStream_t st);
 cudaError_t launch_sinkhorn(const float* l, float* out, int64_t count, int n, int iters, cudaStream_t st);

@@ -143,3 +143,36 @@ def test_mid_bf16_decode_matches_oracle():
         assert L.loop_device_status() == 0
     finally:
         L.loop_model_destroy(g)
+
+
+def test_group9b_decode_matches_oracle():
+    """Decode at the 9B width (hidden 4096, FFN 12288, GQA 32/8 x 128, 32 GLA
+    heads): the decode-only kernels (one-launch mHC site, weight-streaming
+    GEMM, decode attention, GLA step) against the oracle, on a 4-layer group
+    run twice with a 4096-token vocabulary."""
+    w = W.WORKLOADS["probe_decode_b64_ctx4096"]
+    B, S, steps = 2, 32, 2
+    m = dict(w["model"], max_batch=B, max_ctx=S + steps)
+    g = L.loop_model_create(L.make_config(**m), seed=7)
+    try:
+        o = oracle.Model(oracle.make_config(**m), seed=7)
+        tok = seeded.tokens(7, B, S, m["vocab"])
+        nxt = seeded.tokens(7, B, steps, m["vocab"], stream=seeded.S_DECODE_TOKENS)
+        ref = o.prefill(tok)
+        out = torch.empty((B, m["vocab"]), device="cuda")
+        L.loop_prefill(g, tokens=torch.from_numpy(tok).cuda(), out=out)
+        torch.cuda.synchronize()
+        check(out.cpu().numpy(), ref)
+        for t in range(steps):
+            r = o.decode_step(nxt[:, t])
+            L.loop_decode_step(g, torch.from_numpy(np.ascontiguousarray(nxt[:, t])).cuda(), out)
+            torch.cuda.synchronize()
+            check(out.cpu().numpy(), r)
+        for slot in (0, 5):
+            st = torch.empty((B, 32, 128, 128), device="cuda")
+            L.loop_cache_read(g, L.LOOP_KIND_LINEAR, slot, B, 0, st)
+            torch.cuda.synchronize()
+            check(st.cpu().numpy(), o.state(slot, B))
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
