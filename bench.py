@@ -92,6 +92,26 @@ def layer_weight_bytes(m, full: bool) -> int:
     return 2 * (w_in + w_o + 2 * F * H + H * F)
 
 
+def prefill_step_flops(m, B: int, S: int) -> dict:
+    """Tensor FLOPs one prefill step must do: every layer execution's
+    projections (2 x parameters per token), causal attention (QK^T and PV over
+    the keys at or before each query), the chunked linear-attention products
+    at the pages' chunk length (scores, intra- and inter-chunk outputs, state
+    update), and the LM head on the last position of each sequence."""
+    execs = list(range(m["n_prelude"])) + [m["n_prelude"] + j for j in range(m["n_block"])] * m["n_loops"] + \
+        [m["n_prelude"] + m["n_block"] + j for j in range(m["n_coda"])]
+    full = [p % m["group"] == m["full_slot"] for p in execs]
+    T = B * S
+    proj = sum(2 * T * layer_weight_bytes(m, f) // 2 for f in full)
+    d = m["head_dim"]
+    attn = sum(full) * B * m["n_q"] * 4 * d * (S * (S + 1) // 2)
+    C, dl = m["lin_chunk"], m["lin_dim"]
+    gla = (len(full) - sum(full)) * T * m["n_lin"] * (4 * C * dl + 4 * dl * dl)
+    head = 2 * B * m["hidden"] * m["vocab"] if m["io_mode"] == 0 else 0
+    return {"projections": proj, "attention": attn, "linear_attention": gla, "lm_head": head,
+            "total": proj + attn + gla + head}
+
+
 def decode_step_bytes(m, B: int, ctx: int) -> dict:
     """HBM bytes one decode step must move: every layer execution reads its
     weights (the shared block twice), the head reads E, full attention reads
@@ -437,10 +457,18 @@ def main():
             "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak if peak else None,
             "peak_kind": f"{pk_kind} sustained bf16", "traffic": GEMM_TRAFFIC_PER_LAUNCH,
             "traffic_note": "mean DRAM bytes per GEMM launch (ncu); achieved is over all GEMM launches of the steps"}
+    step_roof = None
+    if not decode:
+        fl = prefill_step_flops(m, w["batch"], w["seq"])
+        step_tf = fl["total"] / (r["ms"] / 1e3) / 1e12
+        step_roof = {"bound": "tensor", "achieved": step_tf, "peak": peak, "unit": "TFLOP/s",
+                     "frac": step_tf / peak if peak else None, "peak_kind": f"{pk_kind} sustained bf16",
+                     "flops_per_step": fl}
     line = {"metric": metric, "value": r["value"], "unit": unit, "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": DATA, "config": config, "clocks": r["clocks"],
             "roofline": roof,
+            "step_roofline": step_roof,
             "e2e": {"value": r["e2e_value"], "unit": unit, "h2d_bytes_per_step": r["h2d"],
                     "d2h_bytes_per_step": r["d2h"]},
             "gpu_launches": r["launches"],

@@ -1,24 +1,41 @@
-// Chunked gated linear attention (prefill) on the tensor cores.
+// Gated linear attention: the chunked prefill on the 5th-generation tensor
+// cores (tcgen05) and the one-token decode step.
 //
 // The layer (one of the 3 linear-attention layers of every 4-layer group,
 // "How Does SenseNova-Loop Get More Depth Without More Parameters?", section
 // "How does the hybrid attention pattern work?") keeps a fixed-size state per
-// head: S_t = g_t S_{t-1} + k_t v_t^T, o_t = q_t S_t.  Over a chunk of C = 64
-// tokens with b_t the running sum of log g inside the chunk this is exactly
-//   O   = ((Q K^T) * D) V + diag(exp b) Q S_prev,   D_ts = exp(b_t - b_s) [s <= t]
-//   S'  = exp(b_last) S_prev + K^T (diag(exp(b_last - b)) V).
+// head: S_t = g_t S_{t-1} + k_t v_t^T, o_t = q_t S_t.  Over a tile of T
+// tokens with b_t the running sum of log g inside the tile this is exactly
+//   O  = diag(exp b) Q S_prev + ((Q K^T) * D) V,   D_ts = exp(b_t - b_s) [s <= t]
+//   S' = exp(b_last) S_prev + K^T (diag(exp(b_last - b)) V).
+// The prefill kernel takes T = 128: two of the pages' 64-token chunks, whose
+// joint intra-tile block is the same sum computed in one product (the
+// chunked form is exact for any chunk length), so every product is a full
+// M = 128 tensor-core tile.
 //
-// One CTA (8 warps) owns (sequence, head, 64-column slice of the value
-// dimension) and walks the chunks in order; its 128 x 64 fp32 state slice
-// stays in MMA accumulator registers for the whole sequence (16 rows per
-// warp).  Outputs: warp w computes rows 16 (w % 4) .. + 15 and value columns
-// 32 (w / 4) .. + 31 of the chunk.  Q, K and the V slice of each
-// chunk are staged by TMA (128-byte swizzle, double-buffered).  Products run
-// on bf16 mma.sync m16n8k16 with fp32 accumulation.  The three operands that
-// are not model activations - the state, the decayed scores (Q K^T) * D and
-// the decayed values - enter their products as bf16 hi + lo pairs (~16
-// significant bits), so the chunked form loses no accuracy against the
-// token-by-token recurrence.
+// One CTA per (sequence, head) walks the tiles in order (12 warps):
+//   warp 0      TMA producer: Q, K and V of the tile ([128][128] bf16 each,
+//               two 64-column boxes, 128-byte swizzle), each refilled as soon
+//               as the products that read it are done;
+//   warp 1      one thread issues the tcgen05.mma products:
+//                 P   = Q K^T                       (TMEM, fp32)
+//                 O_x = Q S_prev                    (S as bf16 hi + lo, MN-major)
+//                 R  += K^T V^                      (K read MN-major as A)
+//                 O_a = A V                         (A from TMEM, hi + lo)
+//               where R is the fp32 state, resident in TMEM for the whole
+//               sequence;
+//   warp 2      allocates / frees the 512 TMEM columns;
+//   warps 4-11  each owns one TMEM lane quarter (warp % 4) and one half of
+//               the 128 columns: the decayed scores A = P * D written back
+//               over P as bf16 hi + lo (the A operand of O_a), V^ = diag(exp(
+//               b_last - b)) V as hi + lo in shared memory, the state step
+//               (R -> S_prev hi + lo in shared memory, R *= exp(b_last)), and
+//               the output exp(b_t) O_x + O_a.
+// The three operands that are not model activations (the state, the decayed
+// scores and the decayed values) enter their products as bf16 hi + lo pairs
+// (~16 significant bits), so the chunked form keeps the accuracy of the
+// token-by-token recurrence.  Every mbarrier wait gives up after ~2 s and
+// flags the status word.
 
 #include <cuda.h>
 
@@ -28,257 +45,340 @@ namespace loopk {
 
 namespace {
 
-constexpr int C = 64, DK = 128, DV = 64, WARPS = 8, THREADS = WARPS * 32;
-constexpr int QK_BYTES = C * DK * 2;            // Q or K tile: two boxes [64][64]
-constexpr int V_BYTES = C * DV * 2;             // V slice: one box [64][64]
-constexpr int STAGE_BYTES = 2 * QK_BYTES + V_BYTES;
-constexpr int SS_BYTES = DK * DV * 2;           // bf16 copy of the state slice
-constexpr int SMEM = 2 * STAGE_BYTES + 2 * SS_BYTES + 2 * V_BYTES + 2 * C * 4 + 64 + 1024;
+constexpr int DK = 128;
+constexpr int CT = 128;                       // tokens per tile
+constexpr int TILE = CT * 128 * 2;            // one [128][128] bf16 operand: two boxes [128][64]
+constexpr int THREADS = 384;
+constexpr int OFF_Q = 0, OFF_K = TILE, OFF_V = 2 * TILE, OFF_SHI = 3 * TILE, OFF_SLO = 4 * TILE,
+              OFF_VHI = 5 * TILE, OFF_VLO = 6 * TILE, OFF_B2 = 7 * TILE;
+constexpr int NB2 = 3;                        // gate buffers (tiles t, t + 1 and one in flight)
+enum { B_QF, B_KF, B_VF, B_QE, B_KE, B_VE, B_PF, B_DS, B_OF, B_GR, B_SR, B_VR, B_AR, B_OE, NBARS };
+constexpr int OFF_BAR = OFF_B2 + NB2 * CT * 4;
+constexpr int SMEM = OFF_BAR + NBARS * 8 + 16 + 1024;
+static_assert(SMEM <= 232448, "shared memory per block");
+// TMEM columns: state R, scores P (then A), inter-tile O_x, intra-tile O_a
+constexpr uint32_t T_R = 0, T_P = 128, T_OX = 256, T_OA = 384;
+constexpr uint32_t ID_KK = idesc_bf16_f32(128, 128);               // A, B K-major
+constexpr uint32_t ID_KM = idesc_bf16_f32(128, 128, true);         // B MN-major
+constexpr uint32_t ID_MM = idesc_bf16_f32(128, 128, true, true);   // A, B MN-major
+constexpr float LOG2E = 1.4426950408889634f;
+
+// K-major descriptor of a [128][128] operand, k-step kk (16 columns)
+LOOP_DEV uint64_t kdesc(uint32_t base, int kk) {
+  return smem_desc_sw128(base + (uint32_t)((kk >> 2) * CT * 128 + (kk & 3) * 32), 1024);
+}
+// MN-major descriptor of a [128 k][128 mn] operand, k-step kk (16 rows)
+LOOP_DEV uint64_t mdesc(uint32_t base, int kk) { return smem_desc_sw128_lbo(base + (uint32_t)kk * 2048, TILE / 2, 1024); }
+// TMEM column of the A hi part for k-step kk: each 32-column group of P holds
+// the hi pairs of its 32 keys in its first 16 columns and the lo pairs after
+LOOP_DEV uint32_t a_col(int kk) { return (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)); }
+
+LOOP_DEV void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = pack_bf16x2(x0 - hf.x, x1 - hf.y);
+}
 
 __global__ void __launch_bounds__(THREADS, 1)
-    gla_chunk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                     const __grid_constant__ CUtensorMap tv, const float* __restrict__ gl, float* __restrict__ state,
-                     bf16* __restrict__ out, int S, int nh, int* status) {
+    gla_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                  const __grid_constant__ CUtensorMap tv, const float* __restrict__ gl, float* __restrict__ state,
+                  bf16* __restrict__ out, int S, int nh, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* stage0 = smem;
-  uint8_t* shi = smem + 2 * STAGE_BYTES;
-  uint8_t* slo = shi + SS_BYTES;
-  uint8_t* vhat = slo + SS_BYTES;      // hi part of diag(exp(b_last - b)) V
-  uint8_t* vhat_lo = vhat + V_BYTES;    // and its remainder
-  float* lg = reinterpret_cast<float*>(vhat_lo + V_BYTES);
-  float* bv = lg + C;
-  uint64_t* full = reinterpret_cast<uint64_t*>(bv + C);
+  float* b2s = reinterpret_cast<float*>(smem + OFF_B2);  // [NB2][CT] running log2 gates
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + NBARS);
 
-  const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3, mi = lane >> 3, ri = lane & 7;
-  const int nch = (S + C - 1) / C;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = (S + CT - 1) / CT;
   const int row0 = (b * nh + h) * S;  // first row of this head in the [B nh S][128] views
-  const float* glh = gl + (int64_t)(b * nh + h) * S;
-  float* st = state + (int64_t)(b * nh + h) * DK * 128 + slice * DV;
+  const int64_t bh = (int64_t)b * nh + h;
 
-  if (tid == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBARS; ++i) mbar_init(&bar[i], i >= B_SR ? 8u : 1u);
     fence_mbar_init();
   }
+  if (warp == 2) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
   __syncthreads();
-  auto issue = [&](int c) {
-    uint8_t* sg = stage0 + (c & 1) * STAGE_BYTES;
-    uint64_t* bar = &full[c & 1];
-    const int row = row0 + c * C;
-    mbar_expect_tx(bar, STAGE_BYTES);
-    tma_load_2d(sg, &tq, bar, 0, row);
-    tma_load_2d(sg + QK_BYTES / 2, &tq, bar, 64, row);
-    tma_load_2d(sg + QK_BYTES, &tk, bar, 0, row);
-    tma_load_2d(sg + QK_BYTES + QK_BYTES / 2, &tk, bar, 64, row);
-    tma_load_2d(sg + 2 * QK_BYTES, &tv, bar, slice * DV, row);
-  };
-  if (tid == 0) {
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t su = smem_u32(smem);
+
+  if (warp == 0 && lane == 0) {
     prefetch_tmap(&tq);
     prefetch_tmap(&tk);
     prefetch_tmap(&tv);
-    issue(0);
-    if (nch > 1) issue(1);
-  }
-
-  // state slice: warp w owns rows 16w .. 16w + 15 (one m16 tile) x 64 columns
-  float acc[8][4];
+    const CUtensorMap* maps[3] = {&tq, &tk, &tv};
+    for (int c = 0; c < nch; ++c) {
+      const int row = row0 + c * CT;
+      bool ok = true;
+      for (int o = 0; o < 3 && ok; ++o) {  // Q, K, V in the order the products release them
+        if (c > 0 && !mbar_wait(&bar[B_QE + o], (c - 1) & 1, status, STATUS_WAIT_PRODUCER)) { ok = false; break; }
+        uint8_t* dst = smem + o * TILE;
+        mbar_expect_tx(&bar[B_QF + o], TILE);
+        tma_load_2d(dst, maps[o], &bar[B_QF + o], 0, row);
+        tma_load_2d(dst + TILE / 2, maps[o], &bar[B_QF + o], 64, row);
+      }
+      if (!ok) break;
+    }
+  } else if (warp == 1 && lane == 0) {
+    auto scores = [&]() {
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    const int r = warp * 16 + g, c = nt * 8 + 2 * t;
-    acc[nt][0] = st[(int64_t)r * 128 + c];
-    acc[nt][1] = st[(int64_t)r * 128 + c + 1];
-    acc[nt][2] = st[(int64_t)(r + 8) * 128 + c];
-    acc[nt][3] = st[(int64_t)(r + 8) * 128 + c + 1];
-  }
+      for (int kk = 0; kk < 8; ++kk) tc_mma_f16(tmem + T_P, kdesc(su + OFF_Q, kk), kdesc(su + OFF_K, kk), ID_KK, kk > 0);
+      tc_commit(&bar[B_PF]);
+    };
+    bool ok = mbar_wait(&bar[B_QF], 0, status, STATUS_WAIT_MMA) && mbar_wait(&bar[B_KF], 0, status, STATUS_WAIT_MMA);
+    if (ok) {
+      tc_fence_after();
+      scores();
+    }
+    for (int c = 0; c < nch && ok; ++c) {
+      const uint32_t par = c & 1;
+      // O_x = Q S_prev once the state step has written S_prev and the last
+      // tile's outputs have been read
+      ok = mbar_wait(&bar[B_SR], par, status, STATUS_WAIT_MMA) &&
+           (c == 0 || mbar_wait(&bar[B_OE], (c - 1) & 1, status, STATUS_WAIT_MMA));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) tc_mma_f16(tmem + T_OX, kdesc(su + OFF_Q, kk), mdesc(su + OFF_SHI, kk), ID_KM, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) tc_mma_f16(tmem + T_OX, kdesc(su + OFF_Q, kk), mdesc(su + OFF_SLO, kk), ID_KM, 1u);
+      tc_commit(&bar[B_QE]);
+      // R += K^T V^
+      if (!mbar_wait(&bar[B_VR], par, status, STATUS_WAIT_MMA)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) tc_mma_f16(tmem + T_R, mdesc(su + OFF_K, kk), mdesc(su + OFF_VHI, kk), ID_MM, 1u);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) tc_mma_f16(tmem + T_R, mdesc(su + OFF_K, kk), mdesc(su + OFF_VLO, kk), ID_MM, 1u);
+      tc_commit(&bar[B_DS]);
+      tc_commit(&bar[B_KE]);
+      // O_a = A V, A from TMEM
+      ok = mbar_wait(&bar[B_AR], par, status, STATUS_WAIT_MMA) && mbar_wait(&bar[B_VF], par, status, STATUS_WAIT_MMA);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) tc_mma_f16_ts(tmem + T_OA, tmem + T_P + a_col(kk), mdesc(su + OFF_V, kk), ID_KM, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) tc_mma_f16_ts(tmem + T_OA, tmem + T_P + a_col(kk) + 16, mdesc(su + OFF_V, kk), ID_KM, 1u);
+      tc_commit(&bar[B_OF]);
+      tc_commit(&bar[B_VE]);
+      if (c + 1 < nch) {
+        // the next scores overwrite A: wait for this tile's products first
+        ok = mbar_wait(&bar[B_OF], par, status, STATUS_WAIT_MMA) &&
+             mbar_wait(&bar[B_QF], (c + 1) & 1, status, STATUS_WAIT_MMA) &&
+             mbar_wait(&bar[B_KF], (c + 1) & 1, status, STATUS_WAIT_MMA);
+        if (!ok) break;
+        tc_fence_after();
+        scores();
+      }
+    }
+  } else if (warp >= 4) {
+    const int ew = warp - 4;
+    const int quarter = warp & 3;     // TMEM lanes 32 quarter .. (fixed by the warp's rank)
+    const int cb = 64 * (ew >> 2);    // this warp's column half
+    const int r = 32 * quarter + lane;  // the row this thread owns: token t, key s or state row
+    const uint32_t lo_lane = (uint32_t)(32 * quarter) << 16;
+    const float* glh = gl + bh * S;
+    bool ok = true;
 
-  const uint32_t shi_u = smem_u32(shi), slo_u = smem_u32(slo), vhat_u = smem_u32(vhat),
-                 vlo_u = smem_u32(vhat_lo);
-  const int rg = warp & 3, ch = warp >> 2;  // output phase: rows 16 rg .., value columns 32 ch ..
-  for (int c = 0; c < nch; ++c) {
-    const int c0 = c * C;
-    const int valid = min(C, S - c0);
-    // gates of this chunk (0 past the end) and their running sums b
-    if (tid < C) lg[tid] = tid < valid ? glh[c0 + tid] : 0.f;
-    const bool ok = mbar_wait(&full[c & 1], (c >> 1) & 1, status, STATUS_WAIT_OTHER);
-    if (__syncthreads_or(!ok)) break;
-    if (warp == 0) {
-      const float x0 = lg[2 * lane], x1 = lg[2 * lane + 1];
-      const float pair = x0 + x1;
-      float inc = pair;
+    // running sums of the log gates of tile j, in log2 units (0 past the end)
+    auto gates = [&](int j) -> bool {
+      if (ew != 0) return true;
+      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bar[B_SR], (j - 1) & 1, status, STATUS_WAIT_EPILOGUE)))
+        return false;  // every warp has read the gate buffer this one reuses
+      const int c0 = j * CT, valid = min(CT, S - c0);
+      float x[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) x[i] = 4 * lane + i < valid ? glh[c0 + 4 * lane + i] : 0.f;
+      x[1] += x[0];
+      x[2] += x[1];
+      x[3] += x[2];
+      float inc = x[3];
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float y = __shfl_up_sync(0xffffffffu, inc, o);
         if (lane >= o) inc += y;
       }
-      const float ex = inc - pair;
-      bv[2 * lane] = ex + x0;
-      bv[2 * lane + 1] = inc;
-    }
-    // current state as bf16 hi + lo, row-major [dk][64] with the 128-byte swizzle
+      const float ex = inc - x[3];
+      float* dst = b2s + (j % NB2) * CT + 4 * lane;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int r = warp * 16 + g + 8 * hf;
-        const float x0 = acc[nt][2 * hf], x1 = acc[nt][2 * hf + 1];
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
-        const float2 hf2 = __bfloat1622float2(hi);
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(x0 - hf2.x, x1 - hf2.y);
-        const uint32_t off = (uint32_t)(r * 128 + ((nt ^ (r & 7)) << 4) + 4 * t);
-        *reinterpret_cast<__nv_bfloat162*>(shi + off) = hi;
-        *reinterpret_cast<__nv_bfloat162*>(slo + off) = lo;
+      for (int i = 0; i < 4; ++i) dst[i] = (ex + x[i]) * LOG2E;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_GR]);
+      return true;
+    };
+    // state step for tile j: S_prev = R (the initial state for j = 0) into
+    // shared memory as hi + lo, then R = exp(b_last) S_prev
+    auto state_step = [&](int j) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_GR], j & 1, status, STATUS_WAIT_EPILOGUE))) return false;
+      if (j >= 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_DS], (j - 1) & 1, status, STATUS_WAIT_EPILOGUE))) return false;
+        tc_fence_after();
       }
-    __syncthreads();
-    const float b_last = bv[C - 1];
-    uint8_t* sg = stage0 + (c & 1) * STAGE_BYTES;
-    const uint32_t q_u = smem_u32(sg), k_u = q_u + QK_BYTES, v_u = q_u + 2 * QK_BYTES;
-    // V-hat = diag(exp(b_last - b)) V as hi + lo, zero past the end of the sequence
-    for (int ci = tid; ci < C * 8; ci += THREADS) {
-      const int r = ci >> 3, chk = ci & 7;
-      const uint32_t off = (uint32_t)(r * 128 + ((chk ^ (r & 7)) << 4));
-      const float f = r < valid ? __expf(b_last - bv[r]) : 0.f;
-      uint4 u = *reinterpret_cast<const uint4*>(sg + 2 * QK_BYTES + off);
-      uint4 w;
-      __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&u);
-      __nv_bfloat162* pl = reinterpret_cast<__nv_bfloat162*>(&w);
+      const float dl = ex2(b2s[(j % NB2) * CT + CT - 1]);
+      const float* src = state + (bh * DK + r) * 128;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        const int col = cb + 32 * hh;
+        float s[32];
+        if (j == 0) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 x = __bfloat1622float2(p[e]);
-        const float y0 = x.x * f, y1 = x.y * f;
-        p[e] = __floats2bfloat162_rn(y0, y1);
-        const float2 hi = __bfloat1622float2(p[e]);
-        pl[e] = __floats2bfloat162_rn(y0 - hi.x, y1 - hi.y);
+          for (int i = 0; i < 8; ++i) {
+            const float4 v = reinterpret_cast<const float4*>(src + col)[i];
+            s[4 * i] = v.x;
+            s[4 * i + 1] = v.y;
+            s[4 * i + 2] = v.z;
+            s[4 * i + 3] = v.w;
+          }
+        } else {
+          tmem_ld32(tmem + T_R + lo_lane + col, s);
+          tc_wait_ld();
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint4 hi, lo;
+          split_pack(s[8 * ch], s[8 * ch + 1], hi.x, lo.x);
+          split_pack(s[8 * ch + 2], s[8 * ch + 3], hi.y, lo.y);
+          split_pack(s[8 * ch + 4], s[8 * ch + 5], hi.z, lo.z);
+          split_pack(s[8 * ch + 6], s[8 * ch + 7], hi.w, lo.w);
+          const uint32_t off = sw(r, col / 8 + ch, CT);
+          *reinterpret_cast<uint4*>(smem + OFF_SHI + off) = hi;
+          *reinterpret_cast<uint4*>(smem + OFF_SLO + off) = lo;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[i] *= dl;
+        tmem_st32(tmem + T_R + lo_lane + col, s);
       }
-      *reinterpret_cast<uint4*>(vhat + off) = u;
-      *reinterpret_cast<uint4*>(vhat_lo + off) = w;
-    }
-    __syncthreads();
+      tc_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_SR]);
+      return true;
+    };
+    // the final state of the sequence back to global memory
+    auto state_out = [&](int last) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_DS], last & 1, status, STATUS_WAIT_EPILOGUE))) return false;
+      tc_fence_after();
+      float* dst = state + (bh * DK + r) * 128;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        const int col = cb + 32 * hh;
+        float s[32];
+        tmem_ld32(tmem + T_R + lo_lane + col, s);
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          reinterpret_cast<float4*>(dst + col)[i] = make_float4(s[4 * i], s[4 * i + 1], s[4 * i + 2], s[4 * i + 3]);
+      }
+      return true;
+    };
+    // V^ = diag(exp(b_last - b)) V as hi + lo, zero past the end of the sequence
+    auto vhat = [&](int j) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_VF], j & 1, status, STATUS_WAIT_EPILOGUE))) return false;
+      const float* bb = b2s + (j % NB2) * CT;
+      const int valid = min(CT, S - j * CT);
+      const float w = r < valid ? ex2(bb[CT - 1] - bb[r]) : 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t off = sw(r, cb / 8 + ch, CT);
+        const uint4 u = *reinterpret_cast<const uint4*>(smem + OFF_V + off);
+        const uint32_t in[4] = {u.x, u.y, u.z, u.w};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[e]));
+          split_pack(x.x * w, x.y * w, hi[e], lo[e]);
+        }
+        *reinterpret_cast<uint4*>(smem + OFF_VHI + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(smem + OFF_VLO + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_VR]);
+      return true;
+    };
+    // A = (Q K^T) * D over P, as bf16 hi + lo pairs (row t = r, keys cb ..)
+    auto decayed_scores = [&](int j) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_PF], j & 1, status, STATUS_WAIT_EPILOGUE))) return false;
+      tc_fence_after();
+      const float* bb = b2s + (j % NB2) * CT;
+      const int valid = min(CT, S - j * CT);
+      const float bt = bb[r];
+      const bool row_ok = r < valid;
+#pragma unroll 1
+      for (int g = 0; g < 2; ++g) {
+        const int col = cb + 32 * g;
+        float p[32];
+        tmem_ld32(tmem + T_P + lo_lane + col, p);
+        tc_wait_ld();
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int s0 = col + 2 * i;
+          const float x0 = (row_ok && s0 <= r) ? p[2 * i] * ex2(bt - bb[s0]) : 0.f;
+          const float x1 = (row_ok && s0 + 1 <= r) ? p[2 * i + 1] * ex2(bt - bb[s0 + 1]) : 0.f;
+          split_pack(x0, x1, hi[i], lo[i]);
+        }
+        tmem_st16(tmem + T_P + lo_lane + col, hi);
+        tmem_st16(tmem + T_P + lo_lane + col + 16, lo);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_AR]);
+      return true;
+    };
+    // o_t = exp(b_t) O_x + O_a for the valid rows of tile c
+    auto output = [&](int c) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_OF], c & 1, status, STATUS_WAIT_EPILOGUE))) return false;
+      tc_fence_after();
+      const int c0 = c * CT, valid = min(CT, S - c0);
+      const float et = ex2(b2s[(c % NB2) * CT + r]);
+      bf16* dst = out + ((int64_t)b * S + c0 + r) * ((int64_t)nh * 128) + h * 128;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        const int col = cb + 32 * hh;
+        float x[32], a[32];
+        tmem_ld32(tmem + T_OX + lo_lane + col, x);
+        tmem_ld32(tmem + T_OA + lo_lane + col, a);
+        tc_wait_ld();
+        if (r < valid) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = fmaf(et, x[i], a[i]);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + col);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            d4[i] = make_uint4(pack_bf16x2(x[8 * i], x[8 * i + 1]), pack_bf16x2(x[8 * i + 2], x[8 * i + 3]),
+                               pack_bf16x2(x[8 * i + 4], x[8 * i + 5]), pack_bf16x2(x[8 * i + 6], x[8 * i + 7]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_OE]);
+      return true;
+    };
 
-    // ---- outputs: rows 16 rg .. 16 rg + 15, value columns 32 ch .. 32 ch + 31 ----
-    {
-      uint32_t qf[8][4];
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        ldsm_x4(q_u + sw(rg * 16 + (mi & 1) * 8 + ri, kk * 2 + (mi >> 1), C), qf[kk][0], qf[kk][1], qf[kk][2],
-                qf[kk][3]);
-      float a[8][4];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) a[i][0] = a[i][1] = a[i][2] = a[i][3] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-#pragma unroll
-        for (int nt = 0; nt < 8; nt += 2) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(k_u + sw(nt * 8 + (mi >> 1) * 8 + ri, kk * 2 + (mi & 1), C), b0, b1, b2, b3);
-          mma_bf16(a[nt], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
-          mma_bf16(a[nt + 1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
-        }
-      const int tq0 = rg * 16 + g, tq1 = tq0 + 8;
-      const float bt0 = bv[tq0], bt1 = bv[tq1];
-      uint32_t pa[8][2], pl[8][2];  // (Q K^T) * D as bf16 hi + lo
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        float d[4];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int sk = nt * 8 + 2 * t + e;
-          const float bs = bv[sk];
-          d[e] = (sk <= tq0 && sk < valid) ? __expf(bt0 - bs) : 0.f;
-          d[2 + e] = (sk <= tq1 && sk < valid) ? __expf(bt1 - bs) : 0.f;
-        }
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const float x0 = a[nt][2 * hf] * d[2 * hf], x1 = a[nt][2 * hf + 1] * d[2 * hf + 1];
-          const __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
-          const float2 h2 = __bfloat1622float2(hi);
-          pa[nt][hf] = *reinterpret_cast<const uint32_t*>(&hi);
-          pl[nt][hf] = pack_bf16x2(x0 - h2.x, x1 - h2.y);
-        }
-      }
-      // inter-chunk first: o = exp(b_t) Q S_prev (S as hi + lo), then the
-      // intra-chunk (A * D) V accumulates onto it
-      float o[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-#pragma unroll
-        for (int nt = 0; nt < 4; nt += 2) {
-          uint32_t b0, b1, b2, b3;
-          const uint32_t off = sw(kk * 16 + (mi & 1) * 8 + ri, ch * 4 + nt + (mi >> 1), DK);
-          ldsm_x4_t(shi_u + off, b0, b1, b2, b3);
-          mma_bf16(o[nt], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
-          mma_bf16(o[nt + 1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
-          ldsm_x4_t(slo_u + off, b0, b1, b2, b3);
-          mma_bf16(o[nt], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
-          mma_bf16(o[nt + 1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
-        }
-      const float e0 = __expf(bt0), e1 = __expf(bt1);
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        o[nt][0] *= e0;
-        o[nt][1] *= e0;
-        o[nt][2] *= e1;
-        o[nt][3] *= e1;
-      }
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-        for (int nt = 0; nt < 4; nt += 2) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(v_u + sw(kk * 16 + (mi & 1) * 8 + ri, ch * 4 + nt + (mi >> 1), C), b0, b1, b2, b3);
-          mma_bf16(o[nt], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b0, b1);
-          mma_bf16(o[nt + 1], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b2, b3);
-          mma_bf16(o[nt], pl[2 * kk][0], pl[2 * kk][1], pl[2 * kk + 1][0], pl[2 * kk + 1][1], b0, b1);
-          mma_bf16(o[nt + 1], pl[2 * kk][0], pl[2 * kk][1], pl[2 * kk + 1][0], pl[2 * kk + 1][1], b2, b3);
-        }
-      const int64_t ld = (int64_t)nh * 128;
-      bf16* r0p = out + ((int64_t)b * S + c0 + tq0) * ld + h * 128 + slice * DV + ch * 32;
-      bf16* r1p = out + ((int64_t)b * S + c0 + tq1) * ld + h * 128 + slice * DV + ch * 32;
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const int col = nt * 8 + 2 * t;
-        if (tq0 < valid) *reinterpret_cast<uint32_t*>(r0p + col) = pack_bf16x2(o[nt][0], o[nt][1]);
-        if (tq1 < valid) *reinterpret_cast<uint32_t*>(r1p + col) = pack_bf16x2(o[nt][2], o[nt][3]);
-      }
+    ok = gates(0) && state_step(0) && vhat(0) && decayed_scores(0);
+    for (int c = 0; c < nch && ok; ++c) {
+      if (c + 1 < nch)
+        ok = gates(c + 1) && state_step(c + 1);
+      else
+        ok = state_out(c);
+      ok = ok && output(c);
+      if (ok && c + 1 < nch) ok = vhat(c + 1) && decayed_scores(c + 1);
     }
-    // ---- state update: S = exp(b_last) S + K^T V-hat (rows 16 warp ..) ----
-    {
-      const float dl = __expf(b_last);
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][e] *= dl;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t af[4];
-        ldsm_x4_t(k_u + sw(kk * 16 + (mi >> 1) * 8 + ri, 2 * warp + (mi & 1), C), af[0], af[1], af[2], af[3]);
-#pragma unroll
-        for (int nt = 0; nt < 8; nt += 2) {
-          uint32_t b0, b1, b2, b3;
-          const uint32_t off = sw(kk * 16 + (mi & 1) * 8 + ri, nt + (mi >> 1), C);
-          ldsm_x4_t(vhat_u + off, b0, b1, b2, b3);
-          mma_bf16(acc[nt], af[0], af[1], af[2], af[3], b0, b1);
-          mma_bf16(acc[nt + 1], af[0], af[1], af[2], af[3], b2, b3);
-          ldsm_x4_t(vlo_u + off, b0, b1, b2, b3);
-          mma_bf16(acc[nt], af[0], af[1], af[2], af[3], b0, b1);
-          mma_bf16(acc[nt + 1], af[0], af[1], af[2], af[3], b2, b3);
-        }
-      }
-    }
-    __syncthreads();  // every read of this stage, the state copy and V-hat is done
-    if (tid == 0 && c + 2 < nch) issue(c + 2);
   }
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    const int r = warp * 16 + g, c = nt * 8 + 2 * t;
-    st[(int64_t)r * 128 + c] = acc[nt][0];
-    st[(int64_t)r * 128 + c + 1] = acc[nt][1];
-    st[(int64_t)(r + 8) * 128 + c] = acc[nt][2];
-    st[(int64_t)(r + 8) * 128 + c + 1] = acc[nt][3];
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -348,16 +448,16 @@ cudaError_t launch_gla_chunked(const void* q, const void* k, const void* v, cons
   if (B == 0 || S == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv;
   const int64_t rows = (int64_t)B * nh * S;
-  if (!map_rows128(&mq, q, rows, C) || !map_rows128(&mk, k, rows, C) || !map_rows128(&mv, v, rows, C))
+  if (!map_rows128(&mq, q, rows, CT) || !map_rows128(&mk, k, rows, CT) || !map_rows128(&mv, v, rows, CT))
     return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gla_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    cudaError_t e = cudaFuncSetAttribute(gla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid(128 / DV, (unsigned)nh, (unsigned)B);
-  gla_chunk_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, gl, state, (bf16*)o, S, nh, status_ptr());
+  dim3 grid((unsigned)nh, (unsigned)B);
+  gla_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, gl, state, (bf16*)o, S, nh, status_ptr());
   return cudaGetLastError();
 }
 
