@@ -3,19 +3,22 @@
 // Depth Without More Parameters?", section "How does the hybrid attention
 // pattern work?").
 //
-// One CTA computes 128 queries of one head over key tiles of 128:
-//   warp 0      TMA producer: Q once, then K and V tiles into a 2-slot ring
-//               (128-byte swizzle);
-//   warp 1      one thread issues tcgen05.mma: S_j = Q K_j^T into one of two
-//               128-column TMEM buffers, then O += P_{j-1} V_{j-1} into a
-//               third (P from shared memory as the K-major A operand, V read
-//               in place as an MN-major B operand);
-//   warp 2      allocates / frees TMEM;
-//   warps 4-7   softmax: thread r owns query row r, loads its S row from TMEM,
-//               keeps the running max and sum, writes P (bf16) to shared
-//               memory, and rescales its O row in TMEM only when the max grew
-//               by more than 2^8 since the last rescale (the stale max then
-//               bounds P by 256); at the end O / l is stored.
+// One CTA computes two 128-query tiles (X = 0, 1: queries q0 .. q0 + 255) of
+// one head against the key tiles of 128 both need, sharing each K/V tile:
+//   warp 0      TMA producer: Q of both tiles once, then K and V tiles into a
+//               2-slot ring (128-byte swizzle);
+//   warp 1      allocates TMEM; one lane issues tcgen05.mma, alternating the
+//               tiles so one tile's products run while the other's softmax
+//               does:  S_X = Q_X K_j^T into TMEM, then O_X += P_X V_j with P_X
+//               read from TMEM (it overwrites S_X) and V read in place as an
+//               MN-major B operand;
+//   warps 2-5   softmax of tile 0, warps 6-9 softmax of tile 1: thread r owns
+//               query row r of its tile (TMEM lane r), loads its S row, keeps
+//               the running max and sum, writes P (bf16 pairs) back over S,
+//               and rescales its O row in TMEM only when the max grew by more
+//               than 2^8 since the last rescale (the stale max then bounds P
+//               by 256); at the end O / l is stored.
+// TMEM: S_0 (then P_0) at column 0, S_1 at 128, O_0 at 256, O_1 at 384.
 // Every mbarrier wait is bounded; the whole warp leaves together before any
 // warp-collective TMEM access.
 
@@ -28,12 +31,11 @@ namespace loopk {
 namespace {
 
 constexpr int BQ = 128, BKV = 128, D = 128, NS = 2;
-constexpr int THREADS = 256;
+constexpr int THREADS = 320;             // 2 role warps + 2 softmax warpgroups
 constexpr int Q_BYTES = BQ * D * 2;      // 32 KB: two boxes [128][64]
 constexpr int KV_TILE = BKV * D * 2;     // 32 KB: two boxes [128][64]
-constexpr int P_BYTES = BQ * BKV * 2;    // 32 KB
-constexpr int SMEM = Q_BYTES + NS * 2 * KV_TILE + P_BYTES + 1024 + 256;
-constexpr int TMEM_COLS = 512;           // S buffers at 0 and 128, O at 256
+constexpr int SMEM = 2 * Q_BYTES + NS * 2 * KV_TILE + 1024 + 256;
+constexpr int TMEM_COLS = 512;
 constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, D, true);
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
@@ -50,25 +52,24 @@ __global__ void __launch_bounds__(THREADS, 1)
                     int64_t ctx, float scale_log2, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sq = smem;
-  uint8_t* skv = smem + Q_BYTES;  // slot s: K at skv + 2 s KV_TILE, V after it
-  uint8_t* sp = skv + NS * 2 * KV_TILE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sp + P_BYTES);
+  uint8_t* sq = smem;                 // tile X at sq + X Q_BYTES
+  uint8_t* skv = smem + 2 * Q_BYTES;  // slot s: K at skv + 2 s KV_TILE, V after it
+  uint64_t* bars = reinterpret_cast<uint64_t*>(skv + NS * 2 * KV_TILE);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + NS;
-  uint64_t* s_full = kv_empty + NS;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* o_done = p_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
+  uint64_t* s_full = kv_empty + NS;  // [2] one per query tile
+  uint64_t* p_full = s_full + 2;     // [2]
+  uint64_t* pv_done = p_full + 2;    // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
 
-  const int nqb = (S + BQ - 1) / BQ;
-  const int qb = nqb - 1 - (int)blockIdx.x;  // longest rows first
+  const int npair = (S + 2 * BQ - 1) / (2 * BQ);
+  const int q0 = 2 * BQ * (npair - 1 - (int)blockIdx.x);  // longest rows first
   const int h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / (nq / nkv);
-  const int q0 = qb * BQ;
-  const int ntiles = (min(q0 + BQ, S) - 1) / BKV + 1;
+  // key tiles each query tile needs (0: the second tile is past the end)
+  const int nt[2] = {(min(q0 + BQ, S) - 1) / BKV + 1, q0 + BQ < S ? (min(q0 + 2 * BQ, S) - 1) / BKV + 1 : 0};
+  const int ntiles = max(nt[0], nt[1]);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -77,30 +78,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 4);
+      mbar_init(&pv_done[x], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(o_done, 1);
     fence_mbar_init();
   }
-  if (warp == 2) tmem_alloc(tmem_slot, TMEM_COLS);
+  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_s[2] = {tmem, tmem + 128};
-  const uint32_t t_o = tmem + 256;
 
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tq);
     prefetch_tmap(&tk);
     prefetch_tmap(&tv);
     const int qrow = (b * nq + h) * S + q0;
-    mbar_expect_tx(q_full, Q_BYTES);
-    tma_load_2d(sq, &tq, q_full, 0, qrow);
-    tma_load_2d(sq + Q_BYTES / 2, &tq, q_full, 64, qrow);
+    const int ntq = nt[1] > 0 ? 2 : 1;
+    mbar_expect_tx(q_full, ntq * Q_BYTES);
+    for (int x = 0; x < ntq; ++x) {
+      tma_load_2d(sq + x * Q_BYTES, &tq, q_full, 0, qrow + x * BQ);
+      tma_load_2d(sq + x * Q_BYTES + Q_BYTES / 2, &tq, q_full, 64, qrow + x * BQ);
+    }
     const int64_t krow0 = ((int64_t)b * nkv + kvh) * ctx;
     for (int j = 0; j < ntiles; ++j) {
       const int s = j % NS;
@@ -115,65 +116,84 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_load_2d(vt + KV_TILE / 2, &tv, &kv_full[s], 64, row);
     }
   } else if (warp == 1 && lane == 0) {
-    const uint32_t q_u = smem_u32(sq), p_u = smem_u32(sp), kv_u = smem_u32(skv);
-    bool ok = mbar_wait(q_full, 0, status, STATUS_WAIT_MMA);
-    auto issue_pv = [&](int jj) -> bool {  // O += P_jj V_jj
-      if (!mbar_wait(p_full, jj & 1, status, STATUS_WAIT_MMA)) return false;
+    const uint32_t q_u = smem_u32(sq), kv_u = smem_u32(skv);
+    auto slot = [&](int j) { return kv_u + 2 * (j % NS) * KV_TILE; };
+    // S_X(j) = Q_X K_j^T; P_X of key tile j - 1 must have been consumed
+    auto issue_s = [&](int x, int j) -> bool {
+      if (j >= 1 && !mbar_wait(&pv_done[x], (j - 1) & 1, status, STATUS_WAIT_MMA)) return false;
       tc_fence_after();
-      const uint32_t vt = kv_u + (2 * (jj % NS) + 1) * KV_TILE;
-#pragma unroll
-      for (int kk = 0; kk < BKV / 16; ++kk)
-        tc_mma_f16(t_o, kmajor_desc(p_u, BQ, kk), smem_desc_sw128_lbo(vt + kk * 2048, KV_TILE / 2, 1024), IDESC_PV,
-                   (jj > 0 || kk > 0) ? 1u : 0u);
-      tc_commit(&kv_empty[jj % NS]);
-      tc_commit(o_done);
-      return true;
-    };
-    for (int j = 0; j < ntiles && ok; ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait(&kv_full[j % NS], (j / NS) & 1, status, STATUS_WAIT_MMA)) { ok = false; break; }
-      if (j >= 2 && !mbar_wait(&s_free[sb], ((j - 2) >> 1) & 1, status, STATUS_WAIT_MMA)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t kt = kv_u + 2 * (j % NS) * KV_TILE;
+      const uint32_t kt = slot(j);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        tc_mma_f16(t_s[sb], kmajor_desc(q_u, BQ, kk), kmajor_desc(kt, BKV, kk), IDESC_S, kk > 0 ? 1u : 0u);
-      tc_commit(&s_full[sb]);
-      if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        tc_mma_f16(tmem + 128 * x, kmajor_desc(q_u + x * Q_BYTES, BQ, kk), kmajor_desc(kt, BKV, kk), IDESC_S,
+                   kk > 0 ? 1u : 0u);
+      tc_commit(&s_full[x]);
+      return true;
+    };
+    // O_X += P_X V_j, P_X read from TMEM
+    auto issue_pv = [&](int x, int j) -> bool {
+      if (!mbar_wait(&p_full[x], j & 1, status, STATUS_WAIT_MMA)) return false;
+      tc_fence_after();
+      const uint32_t vt = slot(j) + KV_TILE;
+#pragma unroll
+      for (int kk = 0; kk < BKV / 16; ++kk)
+        tc_mma_f16_ts(tmem + 256 + 128 * x, tmem + 128 * x + 8 * kk,
+                      smem_desc_sw128_lbo(vt + kk * 2048, KV_TILE / 2, 1024), IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+      tc_commit(&pv_done[x]);
+      return true;
+    };
+    auto kv_ready = [&](int j) { return mbar_wait(&kv_full[j % NS], (j / NS) & 1, status, STATUS_WAIT_MMA); };
+    // order: S_0(0) S_1(0), then per key tile j: PV_0(j) S_0(j+1) PV_1(j)
+    // S_1(j+1), so each tile's next scores start as soon as its own P is used
+    bool ok = mbar_wait(q_full, 0, status, STATUS_WAIT_MMA) && kv_ready(0);
+    for (int x = 0; x < 2 && ok; ++x)
+      if (nt[x] > 0) ok = issue_s(x, 0);
+    for (int j = 0; j < ntiles && ok; ++j) {
+      bool next_loaded = false;
+      for (int x = 0; x < 2 && ok; ++x) {
+        if (j >= nt[x]) continue;
+        ok = issue_pv(x, j);
+        if (ok && j + 1 < nt[x]) {
+          if (!next_loaded) ok = next_loaded = kv_ready(j + 1);
+          if (ok) ok = issue_s(x, j + 1);
+        }
+      }
+      if (ok) tc_commit(&kv_empty[j % NS]);
     }
-    if (ok) issue_pv(ntiles - 1);
-  } else if (warp >= 4) {
-    const int quarter = warp & 3;
-    const int r = 32 * quarter + lane;  // query row in the block
-    const int qpos = q0 + r;
+  } else if (warp >= 2) {
+    const int x = (warp - 2) >> 2;    // query tile of this warpgroup
+    const int quarter = warp & 3;     // TMEM lanes 32 quarter .. (fixed by the warp's rank)
+    const int r = 32 * quarter + lane;
+    const int qpos = q0 + BQ * x + r;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    uint8_t* prow = sp;
+    const uint32_t t_s = tmem + 128 * x + lane_off, t_o = tmem + 256 + 128 * x + lane_off;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles && ok; ++j) {
-      const int sb = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (j >> 1) & 1, status, STATUS_WAIT_EPILOGUE));
+    for (int j = 0; j < nt[x] && ok; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1, status, STATUS_WAIT_EPILOGUE));
       if (!ok) break;
       tc_fence_after();
       float sv[BKV];
-#pragma unroll
-      for (int c = 0; c < BKV / 32; ++c) {
-        float v[32];
-        tmem_ld32(t_s[sb] + lane_off + 32 * c, v);
-        tc_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[32 * c + i] = v[i];
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-      const int kbase = j * BKV;
+      tmem_ld32(t_s, *reinterpret_cast<float(*)[32]>(sv));
+      tmem_ld32(t_s + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
+      tmem_ld32(t_s + 64, *reinterpret_cast<float(*)[32]>(sv + 64));
+      tmem_ld32(t_s + 96, *reinterpret_cast<float(*)[32]>(sv + 96));
+      tc_wait_ld();
       float mx = -INFINITY;
+      if (j == nt[x] - 1) {  // the key tile on the diagonal (the only one with keys past some rows)
+        const int kbase = j * BKV;
 #pragma unroll
-      for (int i = 0; i < BKV; ++i) {
-        const float x = (kbase + i <= qpos) ? sv[i] * scale_log2 : -INFINITY;
-        sv[i] = x;
-        mx = fmaxf(mx, x);
+        for (int i = 0; i < BKV; ++i) {
+          const float v = (kbase + i <= qpos) ? sv[i] * scale_log2 : -INFINITY;
+          sv[i] = v;
+          mx = fmaxf(mx, v);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < BKV; ++i) {
+          sv[i] *= scale_log2;
+          mx = fmaxf(mx, sv[i]);
+        }
       }
       float corr = 1.f;
       if (mx > m_ref + RESCALE_THRESHOLD) {
@@ -181,52 +201,42 @@ __global__ void __launch_bounds__(THREADS, 1)
         m_ref = mx;
       }
       float rs = 0.f;
-      uint32_t pk[BKV / 2];
+      float pk[BKV / 2];  // bf16 pairs, as raw bits
 #pragma unroll
       for (int i = 0; i < BKV / 2; ++i) {
         const float p0 = ex2(sv[2 * i] - m_ref), p1 = ex2(sv[2 * i + 1] - m_ref);
         rs += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
+        pk[i] = __uint_as_float(pack_bf16x2(p0, p1));
       }
       l = l * corr + rs;
-      // P_{j-1} V_{j-1} must be done before O is rescaled and P is overwritten
-      if (j >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, status, STATUS_WAIT_EPILOGUE));
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, corr != 1.f)) {
+      // PV of the last tile finished before S_j was computed, so O is stable
+      if (j >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            float v[32];
-            tmem_ld32(t_o + lane_off + 32 * c, v);
-            tc_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(t_o + 32 * c, v);
+          tc_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= corr;
-            tmem_st32(t_o + lane_off + 32 * c, v);
-          }
-          tc_wait_st();
+          for (int i = 0; i < 32; ++i) v[i] *= corr;
+          tmem_st32(t_o + 32 * c, v);
         }
       }
-      // P row r: 16 chunks of 8 keys, 128-byte swizzle, two boxes of 64 keys
-#pragma unroll
-      for (int c = 0; c < BKV / 8; ++c) {
-        const uint32_t off = (uint32_t)((c >> 3) * BQ * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-        *reinterpret_cast<uint4*>(prow + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
+      tmem_st32(t_s, *reinterpret_cast<const float(*)[32]>(pk));
+      tmem_st32(t_s + 32, *reinterpret_cast<const float(*)[32]>(pk + 32));
+      tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[x]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (ntiles - 1) & 1, status, STATUS_WAIT_EPILOGUE));
-    if (ok) {
+    if (ok && nt[x] > 0) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (nt[x] - 1) & 1, status, STATUS_WAIT_EPILOGUE));
+    if (ok && nt[x] > 0) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       bf16* orow = out + ((int64_t)b * S + qpos) * ((int64_t)nq * D) + (int64_t)h * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float v[32];
-        tmem_ld32(t_o + lane_off + 32 * c, v);
+        tmem_ld32(t_o + 32 * c, v);
         tc_wait_ld();
         if (qpos < S) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
@@ -242,7 +252,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -268,7 +278,7 @@ cudaError_t launch_flash_tc(const void* q, const void* K, const void* V, void* o
     attr = true;
   }
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-  dim3 grid((unsigned)((S + BQ - 1) / BQ), (unsigned)nq, (unsigned)B);
+  dim3 grid((unsigned)((S + 2 * BQ - 1) / (2 * BQ)), (unsigned)nq, (unsigned)B);
   flash_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, (bf16*)o, S, nq, nkv, ctx, scale_log2, status_ptr());
   return cudaGetLastError();
 }
