@@ -40,6 +40,45 @@ constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, D, true);
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
+// 2^x on the FMA pipe for both lanes of x (x <= 64): x = n + f with n the
+// nearest integer (1.5 * 2^23 added and removed) and f in [-1/2, 1/2], 2^f by
+// a cubic, and n added to the exponent bits.  The cubic's coefficients are the
+// minimax fit that exp2_poly_fit.py computes; relative error < 7.5e-5.  Inputs
+// below -125 give 2^-125, not 0, so masked scores never take this path.
+constexpr float P2_C0 = 0.9999280571937561f, P2_C1 = 0.6932609677314758f, P2_C2 = 0.2426111251115799f,
+                P2_C3 = 0.0551716685295105f;
+LOOP_DEV float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = fadd2(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = fadd2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(make_float2(P2_C3, P2_C3), f, make_float2(P2_C2, P2_C2));
+  p = ffma2(p, f, make_float2(P2_C1, P2_C1));
+  p = ffma2(p, f, make_float2(P2_C0, P2_C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// P for 64 keys (S columns 64 hh ..) of one row: p = 2^(s scale - m_ref) as
+// bf16 pairs into pk, their sum added to rs2.  With POLY one pair in three is
+// evaluated on the FMA pipe so the MUFU unit is not the limit.
+template <bool POLY>
+LOOP_DEV void softmax_half(const float (&sv)[128], int hh, float2 sc, float2 nm, float (&pk)[32], float2& rs2) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int k = 64 * hh + 2 * i;
+    const float2 xx = ffma2(make_float2(sv[k], sv[k + 1]), sc, nm);
+    float2 pp;
+    if (POLY && (i % 3) == 1)
+      pp = exp2_poly2(xx);
+    else
+      pp = make_float2(ex2(xx.x), ex2(xx.y));
+    rs2 = fadd2(rs2, pp);
+    pk[i] = __uint_as_float(pack_bf16x2(pp.x, pp.y));
+  }
+}
+
 // K-major SW128 descriptor of a [rows][128] bf16 tile stored as two boxes of
 // [rows][64]: k-step kk covers columns 16 kk .. 16 kk + 15.
 LOOP_DEV uint64_t kmajor_desc(uint32_t base, int rows, int kk) {
@@ -179,35 +218,35 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_ld32(t_s + 64, *reinterpret_cast<float(*)[32]>(sv + 64));
       tmem_ld32(t_s + 96, *reinterpret_cast<float(*)[32]>(sv + 96));
       tc_wait_ld();
-      float mx = -INFINITY;
-      if (j == nt[x] - 1) {  // the key tile on the diagonal (the only one with keys past some rows)
+      const bool diag = j == nt[x] - 1;  // the key tile on the diagonal (the only one with keys past some rows)
+      if (diag) {
         const int kbase = j * BKV;
 #pragma unroll
-        for (int i = 0; i < BKV; ++i) {
-          const float v = (kbase + i <= qpos) ? sv[i] * scale_log2 : -INFINITY;
-          sv[i] = v;
-          mx = fmaxf(mx, v);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < BKV; ++i) {
-          sv[i] *= scale_log2;
-          mx = fmaxf(mx, sv[i]);
-        }
+        for (int i = 0; i < BKV; ++i)
+          if (kbase + i > qpos) sv[i] = -INFINITY;
       }
+      float mraw = sv[0];
+#pragma unroll
+      for (int i = 1; i < BKV; ++i) mraw = fmaxf(mraw, sv[i]);
+      const float mx = mraw * scale_log2;
       float corr = 1.f;
       if (mx > m_ref + RESCALE_THRESHOLD) {
         corr = ex2(m_ref - mx);  // 0 on the first tile
         m_ref = mx;
       }
-      float rs = 0.f;
-      float pk[BKV / 2];  // bf16 pairs, as raw bits
+      // p = 2^(s scale - m_ref), two lanes per packed FMA and add
+      const float2 sc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
+      float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < BKV / 2; ++i) {
-        const float p0 = ex2(sv[2 * i] - m_ref), p1 = ex2(sv[2 * i + 1] - m_ref);
-        rs += p0 + p1;
-        pk[i] = __uint_as_float(pack_bf16x2(p0, p1));
+      for (int hh = 0; hh < 2; ++hh) {  // P (bf16 pairs) over S columns 32 hh .., all of S already read
+        float pk[32];
+        if (diag)
+          softmax_half<false>(sv, hh, sc, nm, pk, rs2);
+        else
+          softmax_half<true>(sv, hh, sc, nm, pk, rs2);
+        tmem_st32(t_s + 32 * hh, pk);
       }
+      const float rs = rs2.x + rs2.y;
       l = l * corr + rs;
       // PV of the last tile finished before S_j was computed, so O is stable
       if (j >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
@@ -221,8 +260,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_st32(t_o + 32 * c, v);
         }
       }
-      tmem_st32(t_s, *reinterpret_cast<const float(*)[32]>(pk));
-      tmem_st32(t_s + 32, *reinterpret_cast<const float(*)[32]>(pk + 32));
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
