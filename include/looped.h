@@ -129,6 +129,24 @@ LOOP_API int32_t loop_prefill(loop_model* m, const int32_t* d_tokens, const floa
  * LOOP_ERANGE if a sequence would pass max_ctx. */
 LOOP_API int32_t loop_decode_step(loop_model* m, const int32_t* d_tokens, int32_t B, float* d_logits, void* stream);
 
+/* Append k tokens to each of sequences 0..B-1 in one pass: d_tokens int32
+ * [B][k] continues each sequence at its current length, exactly as k calls of
+ * loop_decode_step would, but with all k positions of a sequence in the same
+ * projections (the step a multi-token-prediction or speculative-verification
+ * loop runs; the pages list MTP as available for faster inference: "SenseTime's
+ * SenseNova-Loop-9B Runs Its Own Layers Twice, and It's Open Source", section
+ * "Running it", and "How Does SenseNova-Loop Get More Depth Without More
+ * Parameters?", section "How do you run SenseNova-Loop-9B-Preview?").
+ * d_out fp32 [B][vocab] (last appended position) or [B][k][vocab] with
+ * LOOP_ALL_POSITIONS.  Appends k KV positions per full-attention execution,
+ * advances every linear-attention state by k tokens, then adds k to each
+ * sequence length.  TOKENS_TO_LOGITS models only (LOOP_EINVAL otherwise);
+ * LOOP_ERANGE if a sequence would pass max_ctx, B > max_batch, or B * k
+ * exceeds the model's per-call token budget (max(max_ctx, min(max_batch *
+ * max_ctx, 65536)) tokens). */
+LOOP_API int32_t loop_extend(loop_model* m, const int32_t* d_tokens, int32_t B, int32_t k, float* d_out,
+                             uint32_t flags, void* stream);
+
 /* Sinkhorn projection of `count` n x n matrices (fp32, row-major, device):
  * P = exp(L - max L) with the library's fixed exponential (Cody-Waite
  * reduction and a degree-7 Taylor polynomial, fused multiply-adds), then

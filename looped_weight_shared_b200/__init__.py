@@ -26,7 +26,7 @@ API = ("loop_num_exec", "loop_schedule", "loop_num_weights", "loop_model_create"
        "loop_decode_step", "mhc_sinkhorn", "loop_model_destroy", "loop_seq_len", "loop_cache_read",
        "loop_weight_read", "loop_device_status", "loop_clear_device_status", "loop_last_error",
        "loop_gemm_bf16", "loop_set_timing", "loop_timing_read", "loop_launch_count", "mhc_prologue",
-       "mhc_prologue_noalloc", "loop_selftest_timeout")
+       "mhc_prologue_noalloc", "loop_selftest_timeout", "loop_extend")
 
 
 class loop_config(C.Structure):
@@ -68,6 +68,7 @@ def lib():
             "loop_model_create": (i32, [P(loop_config), vp, u64, P(vp)]),
             "loop_prefill": (i32, [vp, vp, vp, i32, i32, vp, u32, vp]),
             "loop_decode_step": (i32, [vp, vp, i32, vp, vp]),
+            "loop_extend": (i32, [vp, vp, i32, i32, vp, u32, vp]),
             "mhc_sinkhorn": (i32, [vp, vp, i32, i32, i32, vp]),
             "loop_model_destroy": (None, [vp]),
             "loop_seq_len": (i32, [vp, i32]),
@@ -159,6 +160,14 @@ def loop_decode_step(model: int, tokens, logits, stream=None) -> None:
     """tokens: int32 cuda [B]; logits: fp32 cuda [B, vocab]."""
     _check("loop_decode_step", lib().loop_decode_step(C.c_void_p(model), _ptr(tokens), int(tokens.shape[0]),
                                                       _ptr(logits), _stream(stream)))
+
+
+def loop_extend(model: int, tokens, out, flags: int = 0, stream=None) -> None:
+    """tokens: int32 cuda [B, k] appended to each sequence; out: fp32 cuda
+    [B, vocab] (last appended position) or [B, k, vocab] with LOOP_ALL_POSITIONS."""
+    B, k = int(tokens.shape[0]), int(tokens.shape[1])
+    _check("loop_extend", lib().loop_extend(C.c_void_p(model), _ptr(tokens), B, k, _ptr(out), flags,
+                                            _stream(stream)))
 
 
 def mhc_sinkhorn(logits, out, iters: int = 20, stream=None) -> None:

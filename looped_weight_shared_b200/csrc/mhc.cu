@@ -641,9 +641,9 @@ cudaError_t launch_weight_to_f32(const void* src, bool bf, int64_t rows, int64_t
   return cudaGetLastError();
 }
 
-__global__ void advance_kernel(int32_t* len, int B) {
+__global__ void advance_kernel(int32_t* len, int B, int by) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < B) len[b] += 1;
+  if (b < B) len[b] += by;
 }
 __global__ void set_len_kernel(int32_t* len, int B, int S) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
@@ -653,8 +653,8 @@ cudaError_t launch_set_len(int32_t* len, int B, int S, cudaStream_t st) {
   set_len_kernel<<<(B + 127) / 128, 128, 0, st>>>(len, B, S);
   return cudaGetLastError();
 }
-cudaError_t launch_advance(int32_t* len, int B, cudaStream_t st) {
-  advance_kernel<<<(B + 127) / 128, 128, 0, st>>>(len, B);
+cudaError_t launch_advance(int32_t* len, int B, cudaStream_t st, int by) {
+  advance_kernel<<<(B + 127) / 128, 128, 0, st>>>(len, B, by);
   return cudaGetLastError();
 }
 

@@ -461,7 +461,7 @@ cudaError_t attention(Model& m, const void* Kc, const void* Vc, int B, int S, co
                                      m.w.dec_attn, st);
     });
   }
-  if (bf && S > 1 && flash_tc_supported(c.head_dim, c.n_q, c.n_kv))  // a prefill: every sequence starts at 0
+  if (bf && S > 1 && !m.extending && flash_tc_supported(c.head_dim, c.n_q, c.n_kv))  // a prefill: every sequence starts at 0
     return timed(m, LOOP_K_ATTENTION, flops, 1, st, [&] {
       return launch_flash_tc(m.w.q, Kc, Vc, m.w.o, B, S, c.n_q, c.n_kv, c.max_ctx, st);
     });
@@ -680,6 +680,28 @@ int32_t loop_decode_step(loop_model* mp, const int32_t* d_tokens, int32_t B, flo
   if (rc != LOOP_OK) return rc;
   LOOP_CU(timed(m, LOOP_K_OTHER, 0.0, 1, st, [&] { return launch_advance(m.d_seq_len, B, st); }));
   for (int b = 0; b < B; ++b) m.seq_len[b] += 1;
+  return LOOP_OK;
+}
+
+int32_t loop_extend(loop_model* mp, const int32_t* d_tokens, int32_t B, int32_t k, float* d_out, uint32_t flags,
+                    void* stream) {
+  if (!mp || !d_tokens || !d_out) return fail(LOOP_EINVAL, "NULL argument");
+  Model& m = mp->m;
+  if (m.c.io_mode != LOOP_TOKENS_TO_LOGITS) return fail(LOOP_EINVAL, "extend needs TOKENS_TO_LOGITS");
+  if (B <= 0 || k <= 0) return fail(LOOP_EINVAL, "B and k must be positive");
+  if (B > m.c.max_batch) return fail(LOOP_ERANGE, "B > max_batch");
+  if ((int64_t)B * k > m.w.t_max) return fail(LOOP_ERANGE, "B * k exceeds the per-call token budget");
+  for (int b = 0; b < B; ++b)
+    if ((int64_t)m.seq_len[b] + k > m.c.max_ctx) return fail(LOOP_ERANGE, "sequence would pass max_ctx");
+  cudaStream_t st = (cudaStream_t)stream;
+  // the positions of sequence b are seq_len[b] .. seq_len[b] + k - 1: every kernel takes
+  // its start from d_seq_len, and attention uses the kernel that honours per-sequence starts
+  m.extending = true;
+  const int32_t rc = forward(m, d_tokens, nullptr, 0, B, k, m.d_seq_len, d_out, flags, false, st);
+  m.extending = false;
+  if (rc != LOOP_OK) return rc;
+  LOOP_CU(timed(m, LOOP_K_OTHER, 0.0, 1, st, [&] { return launch_advance(m.d_seq_len, B, st, k); }));
+  for (int b = 0; b < B; ++b) m.seq_len[b] += k;
   return LOOP_OK;
 }
 

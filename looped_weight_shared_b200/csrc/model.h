@@ -112,6 +112,7 @@ struct Model {
   std::vector<void*> allocs;
   bool use_tc = false;          // tcgen05 path for bf16 projections
   bool decoding = false;        // inside loop_decode_step: projections use the decode GEMM
+  bool extending = false;       // inside loop_extend: sequences start past 0 (no prefill-only attention)
 };
 
 bool bf16_model(const Model& m);
@@ -162,7 +163,7 @@ cudaError_t launch_gla_recurrent(const void* q, const void* k, const void* v, co
 cudaError_t launch_rope_table(float2* tab, int64_t ctx, int hd, double base, cudaStream_t st);
 cudaError_t launch_cache_to_f32(const void* src, bool bf16, int B, int nkv, int64_t ctx, int len, int hd,
                                 float* dst, cudaStream_t st);
-cudaError_t launch_advance(int32_t* seq_len, int B, cudaStream_t st);
+cudaError_t launch_advance(int32_t* seq_len, int B, cudaStream_t st, int by = 1);
 cudaError_t launch_selftest_timeout(uint64_t limit_ns, int* result, cudaStream_t st);
 cudaError_t launch_set_len(int32_t* seq_len, int B, int S, cudaStream_t st);
 cudaError_t launch_weight_to_f32(const void* src, bool bf16, int64_t rows, int64_t cols, int64_t src_row0,

@@ -176,3 +176,36 @@ def test_group9b_decode_matches_oracle():
         assert L.loop_device_status() == 0
     finally:
         L.loop_model_destroy(g)
+
+
+def test_mid_bf16_extend_matches_decode_steps():
+    """loop_extend on the bf16 tensor-core path: 130 appended tokens span a
+    full 128-token GLA tile plus a ragged one (the chunked kernel resuming from
+    a non-zero state) and attention with keys before the new positions."""
+    B, S, k = 2, 70, 130
+    m = dict(W.model_config("tiny_fp32", **MID), max_batch=B, max_ctx=S + k + 1)
+    g = L.loop_model_create(L.make_config(**m), seed=8)
+    try:
+        o = oracle.Model(oracle.make_config(**m), seed=8)
+        tok = seeded.tokens(8, B, S, m["vocab"])
+        o.prefill(tok)
+        L.loop_prefill(g, tokens=torch.from_numpy(tok).cuda(), out=torch.empty((B, m["vocab"]), device="cuda"))
+        ext = seeded.tokens(8, B, k + 1, m["vocab"], stream=seeded.S_DECODE_TOKENS)
+        ref = np.stack([o.decode_step(ext[:, t]) for t in range(k)], axis=1)
+        out = torch.empty((B, k, m["vocab"]), device="cuda")
+        L.loop_extend(g, torch.from_numpy(np.ascontiguousarray(ext[:, :k])).cuda(), out, flags=L.LOOP_ALL_POSITIONS)
+        torch.cuda.synchronize()
+        check(out.cpu().numpy(), ref)
+        r = o.decode_step(ext[:, k])
+        d = torch.empty((B, m["vocab"]), device="cuda")
+        L.loop_decode_step(g, torch.from_numpy(np.ascontiguousarray(ext[:, k])).cuda(), d)
+        torch.cuda.synchronize()
+        check(d.cpu().numpy(), r)
+        for slot in (0, 5):
+            st = torch.empty((B, 4, 128, 128), device="cuda")
+            L.loop_cache_read(g, L.LOOP_KIND_LINEAR, slot, B, 0, st)
+            torch.cuda.synchronize()
+            check(st.cpu().numpy(), o.state(slot, B))
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)

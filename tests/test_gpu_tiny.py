@@ -189,3 +189,66 @@ def test_hidden_mode_matches_oracle():
         assert rel_err(out.cpu().numpy(), ref) < TOL_F32
     finally:
         L.loop_model_destroy(g)
+
+
+@pytest.mark.parametrize("n_loops", [1, 3])
+def test_loop_count_matches_oracle(n_loops):
+    """Loop counts other than the pages' two, B^K(h) with K = 1 and 3: one
+    weight set reused K times and K sets of per-pass caches, against the
+    oracle through prefill, decode and the last linear-attention state."""
+    m = cfg(n_loops=n_loops)
+    g = L.loop_model_create(L.make_config(**m), seed=0)
+    try:
+        o = oracle.Model(oracle.make_config(**m), seed=0)
+        tok = seeded.tokens(12, 2, 40, m["vocab"])
+        assert rel_err(gpu_prefill(g, tok, m["vocab"]), o.prefill(tok, all_positions=True)) < TOL_F32
+        nxt = seeded.tokens(12, 2, 2, m["vocab"], stream=seeded.S_DECODE_TOKENS)
+        for t in range(2):
+            r = o.decode_step(nxt[:, t])
+            d = torch.empty((2, m["vocab"]), device="cuda")
+            L.loop_decode_step(g, torch.from_numpy(np.ascontiguousarray(nxt[:, t])).cuda(), d)
+            torch.cuda.synchronize()
+            assert rel_err(d.cpu().numpy(), r) < TOL_F32
+        # prelude, K passes of the block and coda each hold one group: 3 linear executions per group
+        last = 3 * (2 + n_loops) - 1
+        st = torch.empty((2, m["n_lin"], m["lin_dim"], m["lin_dim"]), device="cuda")
+        L.loop_cache_read(g, L.LOOP_KIND_LINEAR, last, 2, 0, st)
+        torch.cuda.synchronize()
+        assert rel_err(st.cpu().numpy(), o.state(last, 2)) < TOL_F32
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
+
+
+@pytest.mark.parametrize("k", [1, 6])
+def test_extend_equals_decode_steps(k):
+    """loop_extend appends k tokens per sequence in one pass; the oracle
+    appends them one decode step at a time: every appended position's logits,
+    the lengths and a following decode step agree."""
+    m = cfg()
+    g = L.loop_model_create(L.make_config(**m), seed=0)
+    try:
+        o = oracle.Model(oracle.make_config(**m), seed=0)
+        B, S = 2, 30
+        tok = seeded.tokens(13, B, S, m["vocab"])
+        o.prefill(tok)
+        gpu_prefill(g, tok, m["vocab"], all_positions=False)
+        ext = seeded.tokens(13, B, k + 1, m["vocab"], stream=seeded.S_DECODE_TOKENS)
+        ref = np.stack([o.decode_step(ext[:, t]) for t in range(k)], axis=1)
+        out = torch.empty((B, k, m["vocab"]), device="cuda")
+        L.loop_extend(g, torch.from_numpy(np.ascontiguousarray(ext[:, :k])).cuda(), out, flags=L.LOOP_ALL_POSITIONS)
+        torch.cuda.synchronize()
+        assert rel_err(out.cpu().numpy(), ref) < TOL_F32
+        assert L.loop_seq_len(g, 0) == S + k and L.loop_seq_len(g, 1) == S + k
+        r = o.decode_step(ext[:, k])
+        d = torch.empty((B, m["vocab"]), device="cuda")
+        L.loop_decode_step(g, torch.from_numpy(np.ascontiguousarray(ext[:, k])).cuda(), d)
+        torch.cuda.synchronize()
+        assert rel_err(d.cpu().numpy(), r) < TOL_F32
+        with pytest.raises(L.LoopError) as e:  # past max_ctx
+            L.loop_extend(g, torch.zeros((B, 160), dtype=torch.int32, device="cuda"),
+                          torch.empty((B, m["vocab"]), device="cuda"))
+        assert e.value.code == L.LOOP_ERANGE
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
