@@ -147,6 +147,20 @@ LOOP_API int32_t loop_decode_step(loop_model* m, const int32_t* d_tokens, int32_
 LOOP_API int32_t loop_extend(loop_model* m, const int32_t* d_tokens, int32_t B, int32_t k, float* d_out,
                              uint32_t flags, void* stream);
 
+/* Prefill sequences b0 .. b0+B-1 from position 0, each with its own length
+ * h_lens[i] (host int32 [B], each in [1, max_ctx]), leaving every other
+ * sequence's caches and length untouched: new requests enter free slots while
+ * the others keep decoding (loop_decode_step handles sequences of different
+ * lengths).  d_tokens int32, the B sequences packed one after another
+ * (sum of h_lens tokens).  d_out fp32 [B][vocab] (each sequence's last
+ * position) or, with LOOP_ALL_POSITIONS, the packed [sum h_lens][vocab].
+ * Each sequence runs as its own pass through the same kernels as
+ * loop_prefill, so its results equal a loop_prefill of that sequence alone.
+ * TOKENS_TO_LOGITS models only; LOOP_ERANGE if b0 + B > max_batch or a length
+ * is outside [1, max_ctx]. */
+LOOP_API int32_t loop_prefill_ragged(loop_model* m, const int32_t* d_tokens, const int32_t* h_lens, int32_t b0,
+                                     int32_t B, float* d_out, uint32_t flags, void* stream);
+
 /* Sinkhorn projection of `count` n x n matrices (fp32, row-major, device):
  * P = exp(L - max L) with the library's fixed exponential (Cody-Waite
  * reduction and a degree-7 Taylor polynomial, fused multiply-adds), then

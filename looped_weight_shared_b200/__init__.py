@@ -26,7 +26,7 @@ API = ("loop_num_exec", "loop_schedule", "loop_num_weights", "loop_model_create"
        "loop_decode_step", "mhc_sinkhorn", "loop_model_destroy", "loop_seq_len", "loop_cache_read",
        "loop_weight_read", "loop_device_status", "loop_clear_device_status", "loop_last_error",
        "loop_gemm_bf16", "loop_set_timing", "loop_timing_read", "loop_launch_count", "mhc_prologue",
-       "mhc_prologue_noalloc", "loop_selftest_timeout", "loop_extend")
+       "mhc_prologue_noalloc", "loop_selftest_timeout", "loop_extend", "loop_prefill_ragged")
 
 
 class loop_config(C.Structure):
@@ -69,6 +69,7 @@ def lib():
             "loop_prefill": (i32, [vp, vp, vp, i32, i32, vp, u32, vp]),
             "loop_decode_step": (i32, [vp, vp, i32, vp, vp]),
             "loop_extend": (i32, [vp, vp, i32, i32, vp, u32, vp]),
+            "loop_prefill_ragged": (i32, [vp, vp, vp, i32, i32, vp, u32, vp]),
             "mhc_sinkhorn": (i32, [vp, vp, i32, i32, i32, vp]),
             "loop_model_destroy": (None, [vp]),
             "loop_seq_len": (i32, [vp, i32]),
@@ -168,6 +169,17 @@ def loop_extend(model: int, tokens, out, flags: int = 0, stream=None) -> None:
     B, k = int(tokens.shape[0]), int(tokens.shape[1])
     _check("loop_extend", lib().loop_extend(C.c_void_p(model), _ptr(tokens), B, k, _ptr(out), flags,
                                             _stream(stream)))
+
+
+def loop_prefill_ragged(model: int, tokens, lens, out, b0: int = 0, flags: int = 0, stream=None) -> None:
+    """tokens: int32 cuda, the sequences packed one after another; lens: their
+    lengths (host ints); prefills sequences b0 .. b0 + len(lens) - 1 only.
+    out: fp32 cuda [len(lens), vocab], or [sum(lens), vocab] with LOOP_ALL_POSITIONS."""
+    import numpy as np
+    arr = np.ascontiguousarray(np.asarray(lens, dtype=np.int32))
+    _check("loop_prefill_ragged", lib().loop_prefill_ragged(C.c_void_p(model), _ptr(tokens),
+                                                            arr.ctypes.data_as(C.c_void_p), int(b0), int(arr.size),
+                                                            _ptr(out), flags, _stream(stream)))
 
 
 def mhc_sinkhorn(logits, out, iters: int = 20, stream=None) -> None:

@@ -705,6 +705,34 @@ int32_t loop_extend(loop_model* mp, const int32_t* d_tokens, int32_t B, int32_t 
   return LOOP_OK;
 }
 
+int32_t loop_prefill_ragged(loop_model* mp, const int32_t* d_tokens, const int32_t* h_lens, int32_t b0, int32_t B,
+                            float* d_out, uint32_t flags, void* stream) {
+  if (!mp || !d_tokens || !h_lens || !d_out) return fail(LOOP_EINVAL, "NULL argument");
+  Model& m = mp->m;
+  const loop_config& c = m.c;
+  if (c.io_mode != LOOP_TOKENS_TO_LOGITS) return fail(LOOP_EINVAL, "ragged prefill needs TOKENS_TO_LOGITS");
+  if (B <= 0 || b0 < 0) return fail(LOOP_EINVAL, "B must be positive and b0 >= 0");
+  if ((int64_t)b0 + B > c.max_batch) return fail(LOOP_ERANGE, "b0 + B > max_batch");
+  for (int i = 0; i < B; ++i)
+    if (h_lens[i] < 1 || h_lens[i] > c.max_ctx) return fail(LOOP_ERANGE, "a length is outside [1, max_ctx]");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t nl = c.n_lin, ld = c.lin_dim;
+  const bool all = flags & LOOP_ALL_POSITIONS;
+  int64_t off = 0;
+  for (int i = 0; i < B; ++i) {
+    const int b = b0 + i, S = h_lens[i];
+    for (int j = 0; j < m.n_lin; ++j)
+      LOOP_CU(cudaMemsetAsync(m.st[j] + (int64_t)b * nl * ld * ld, 0, (size_t)nl * ld * ld * 4, st));
+    float* out = d_out + (all ? off : i) * c.vocab;
+    const int32_t rc = forward(m, d_tokens + off, nullptr, b, 1, S, m.w.zeros, out, flags, false, st);
+    if (rc != LOOP_OK) return rc;
+    LOOP_CU(timed(m, LOOP_K_OTHER, 0.0, 1, st, [&] { return launch_set_len(m.d_seq_len + b, 1, S, st); }));
+    m.seq_len[b] = S;
+    off += S;
+  }
+  return LOOP_OK;
+}
+
 int32_t mhc_sinkhorn(const float* d_logits, float* d_out, int32_t count, int32_t n, int32_t iters, void* stream) {
   if (!d_logits || !d_out) return fail(LOOP_EINVAL, "NULL argument");
   if (count < 0 || n < 1 || n > 8 || iters < 0) return fail(LOOP_EINVAL, "count >= 0, 1 <= n <= 8, iters >= 0");

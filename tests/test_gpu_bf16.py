@@ -209,3 +209,32 @@ def test_mid_bf16_extend_matches_decode_steps():
         assert L.loop_device_status() == 0
     finally:
         L.loop_model_destroy(g)
+
+
+def test_mid_bf16_mixed_length_decode():
+    """Decode over sequences of different lengths on the bf16 tensor-core
+    path (decode attention with per-sequence key counts across several
+    1024-key chunks, the GLA step, the decode GEMM): ragged prefill of 1500,
+    77 and 1030 tokens, then two decode steps, each sequence against its own
+    oracle."""
+    lens = [1500, 77, 1030]
+    m = dict(W.model_config("tiny_fp32", **MID4), max_batch=3, max_ctx=1510)
+    g = L.loop_model_create(L.make_config(**m), seed=9)
+    try:
+        seqs = [seeded.tokens(40 + i, 1, n, m["vocab"])[0] for i, n in enumerate(lens)]
+        os_ = [oracle.Model(oracle.make_config(**m), seed=9) for _ in lens]
+        ref = np.concatenate([o.prefill(s[None, :]) for o, s in zip(os_, seqs)], axis=0)
+        out = torch.empty((3, m["vocab"]), device="cuda")
+        L.loop_prefill_ragged(g, torch.from_numpy(np.concatenate(seqs)).cuda(), lens, out)
+        torch.cuda.synchronize()
+        check(out.cpu().numpy(), ref)
+        nxt = seeded.tokens(50, 2, 3, m["vocab"], stream=seeded.S_DECODE_TOKENS)
+        d = torch.empty((3, m["vocab"]), device="cuda")
+        for t in range(2):
+            L.loop_decode_step(g, torch.from_numpy(np.ascontiguousarray(nxt[t])).cuda(), d)
+            torch.cuda.synchronize()
+            r = np.concatenate([o.decode_step(np.array([x], dtype=np.int32)) for o, x in zip(os_, nxt[t])], axis=0)
+            check(d.cpu().numpy(), r)
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)

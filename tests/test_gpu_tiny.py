@@ -252,3 +252,49 @@ def test_extend_equals_decode_steps(k):
         assert L.loop_device_status() == 0
     finally:
         L.loop_model_destroy(g)
+
+
+def _oracle_decode(os_, toks):
+    return np.concatenate([o.decode_step(np.array([t], dtype=np.int32)) for o, t in zip(os_, toks)], axis=0)
+
+
+def test_ragged_prefill_and_mixed_length_decode():
+    """Continuous batching: sequences of lengths 30, 7 and 19 prefilled into
+    slots 0-2, a decode step over all three at their own lengths, then slot 1
+    refilled with a new 12-token sequence while 0 and 2 keep their caches.
+    Each sequence is checked against its own single-sequence oracle."""
+    m = cfg(max_batch=3)
+    g = L.loop_model_create(L.make_config(**m), seed=0)
+    try:
+        lens = [30, 7, 19]
+        seqs = [seeded.tokens(20 + i, 1, n, m["vocab"])[0] for i, n in enumerate(lens)]
+        os_ = [oracle.Model(oracle.make_config(**m), seed=0) for _ in lens]
+        ref = np.concatenate([o.prefill(s[None, :]) for o, s in zip(os_, seqs)], axis=0)
+        out = torch.empty((3, m["vocab"]), device="cuda")
+        L.loop_prefill_ragged(g, torch.from_numpy(np.concatenate(seqs)).cuda(), lens, out)
+        torch.cuda.synchronize()
+        assert rel_err(out.cpu().numpy(), ref) < TOL_F32
+        assert [L.loop_seq_len(g, b) for b in range(3)] == lens
+        nxt = seeded.tokens(30, 2, 3, m["vocab"], stream=seeded.S_DECODE_TOKENS)
+        d = torch.empty((3, m["vocab"]), device="cuda")
+        L.loop_decode_step(g, torch.from_numpy(np.ascontiguousarray(nxt[0])).cuda(), d)
+        torch.cuda.synchronize()
+        assert rel_err(d.cpu().numpy(), _oracle_decode(os_, nxt[0])) < TOL_F32
+        # slot 1 takes a new request; slots 0 and 2 keep decoding
+        new = seeded.tokens(31, 1, 12, m["vocab"])
+        os_[1] = oracle.Model(oracle.make_config(**m), seed=0)
+        r1 = os_[1].prefill(new)
+        o1 = torch.empty((1, m["vocab"]), device="cuda")
+        L.loop_prefill_ragged(g, torch.from_numpy(new[0]).cuda(), [12], o1, b0=1)
+        torch.cuda.synchronize()
+        assert rel_err(o1.cpu().numpy(), r1) < TOL_F32
+        assert [L.loop_seq_len(g, b) for b in range(3)] == [31, 12, 20]
+        L.loop_decode_step(g, torch.from_numpy(np.ascontiguousarray(nxt[1])).cuda(), d)
+        torch.cuda.synchronize()
+        assert rel_err(d.cpu().numpy(), _oracle_decode(os_, nxt[1])) < TOL_F32
+        with pytest.raises(L.LoopError) as e:
+            L.loop_prefill_ragged(g, torch.from_numpy(new[0]).cuda(), [12], o1, b0=3)
+        assert e.value.code == L.LOOP_ERANGE
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
