@@ -181,6 +181,21 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------- our arm
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's time (every rank gets it); x itself on one rank."""
+    if world <= 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job units per second: all ranks' units over the slowest rank's time."""
+    return units_per_rank * world / (ms / 1e3)
+
+
 def run_ours(a, rank, world, local_rank):
     import torch
     import looped_weight_shared_b200 as L
@@ -244,13 +259,10 @@ def run_ours(a, rank, world, local_rank):
         torch.cuda.synchronize()
     L.loop_set_timing(g, False)
     launches = L.loop_launch_count(g) - launches0
-    ms = ev0.elapsed_time(ev1) / a.steps
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / a.steps, world, dev)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
         torch.distributed.barrier()
-    value = units * world / (ms / 1e3)
+    value = job_throughput(units, world, ms)
     classes = {}
     for ci, cname in enumerate(L.KERNEL_CLASSES):
         tms, n, work = L.loop_timing_read(g, ci)
@@ -299,15 +311,11 @@ def run_ours(a, rank, world, local_rank):
         e2e_step(i)
     ev1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, world, dev)
     L.loop_model_destroy(g)
     return dict(ms=ms, value=value, classes=classes, clocks=clk.summary(), launches=launches, status=status,
-                e2e_ms=e2e_ms, e2e_value=units * world / (e2e_ms / 1e3), h2d=h2d, d2h=d2h, create_s=create_s,
-                units=units)
+                e2e_ms=e2e_ms, e2e_value=job_throughput(units, world, e2e_ms), h2d=h2d, d2h=d2h,
+                create_s=create_s, units=units)
 
 
 def run_decode(a, world, local_rank):
@@ -342,11 +350,7 @@ def run_decode(a, world, local_rank):
             L.loop_decode_step(g, toks[warm + i], out)
         ev1.record(stream)
         torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1) / steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / steps, world, dev)
     # the same steps again with per-launch events, for the per-class split
     L.loop_timing_read(g, 0, reset=True)
     L.loop_set_timing(g, True)
@@ -364,7 +368,7 @@ def run_decode(a, world, local_rank):
     L.loop_model_destroy(g)
     mid_ctx = ctx0 + steps // 2
     by = decode_step_bytes(m, B, mid_ctx)
-    return {"ms": ms, "value": B * world / (ms / 1e3), "bytes": by, "classes": classes, "clocks": clk.summary(),
+    return {"ms": ms, "value": job_throughput(B, world, ms), "bytes": by, "classes": classes, "clocks": clk.summary(),
             "ctx": mid_ctx, "ms_with_launch_events": ms_timed}
 
 
