@@ -73,3 +73,15 @@ def test_create_rejects_without_touching_the_device():
         L.loop_model_create(L.make_config(**m))
     assert e.value.code == L.LOOP_EINVAL
     assert "invalid" in L.last_error()
+
+
+def test_entry_points_reject_null_without_touching_the_device():
+    """Argument errors return a status before any device work, including for
+    the append and ragged-prefill entry points."""
+    lib = L.lib()
+    assert lib.loop_prefill(None, None, None, 1, 1, None, 0, None) == L.LOOP_EINVAL
+    assert lib.loop_decode_step(None, None, 1, None, None) == L.LOOP_EINVAL
+    assert lib.loop_extend(None, None, 1, 1, None, 0, None) == L.LOOP_EINVAL
+    assert lib.loop_prefill_ragged(None, None, None, 0, 1, None, 0, None) == L.LOOP_EINVAL
+    assert "NULL" in L.last_error()
+    assert lib.mhc_sinkhorn(None, None, 1, 2, 20, None) == L.LOOP_EINVAL
