@@ -48,7 +48,7 @@ enum {
   LOOP_ENOMEM = -2,       /* device allocation failed (nothing is leaked)      */
   LOOP_ECUDA = -3,        /* a CUDA call failed                                */
   LOOP_ERANGE = -4,       /* batch > max_batch or context > max_ctx            */
-  LOOP_EUNSUPPORTED = -5, /* valid configuration this build does not run       */
+  LOOP_EUNSUPPORTED = -5, /* valid configuration this library does not run     */
   LOOP_ETIMEOUT = -6      /* a device-side wait gave up (see loop_device_status) */
 };
 
@@ -69,7 +69,7 @@ typedef struct {
   int32_t hidden, ffn, vocab;                  /* [4096, 12288, 248320]; vocab unused for HIDDEN_TO_HIDDEN */
   int32_t n_q, n_kv, head_dim;                 /* full attention, GQA [32, 8, 128] */
   int32_t n_lin, lin_dim, lin_chunk;           /* gated linear attention [32, 128, 64] */
-  int32_t n_streams, sinkhorn_iters;           /* mHC [2, 20]; this build runs n_streams == 2 */
+  int32_t n_streams, sinkhorn_iters;           /* mHC [2, 20]; this library runs n_streams == 2 */
   float rope_base, norm_eps;                   /* [1e4, 1e-6] */
   int32_t dtype;                               /* LOOP_F32 or LOOP_BF16 (mHC parameters are always fp32) */
   int32_t io_mode;                             /* LOOP_TOKENS_TO_LOGITS or LOOP_HIDDEN_TO_HIDDEN */

@@ -58,9 +58,9 @@ bool valid(const loop_config* c) {
   return true;
 }
 
-// What this build runs (valid configurations outside it are LOOP_EUNSUPPORTED).
+// What this library runs (valid configurations outside it are LOOP_EUNSUPPORTED).
 const char* unsupported(const loop_config* c) {
-  if (c->n_streams != 2) return "this build runs n_streams == 2";
+  if (c->n_streams != 2) return "this library runs n_streams == 2";
   if (c->hidden % 4 != 0) return "hidden must be a multiple of 4";
   if ((size_t)9 * c->hidden * 4 > 220 * 1024) return "hidden must be <= 6144 (mHC prologue keeps Phi in shared memory)";
   if (c->ffn % 128 != 0) return "ffn must be a multiple of 128";
