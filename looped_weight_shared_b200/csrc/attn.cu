@@ -268,13 +268,8 @@ cudaError_t launch_attention_decode(const void* q, const void* K, const void* V,
   CUtensorMap mk, mv;
   if (!map_rows128(&mk, K, (int64_t)B * nkv * ctx, DEC_TILE) || !map_rows128(&mv, V, (int64_t)B * nkv * ctx, DEC_TILE))
     return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e =
-        cudaFuncSetAttribute(attn_decode_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_limit(attn_decode_partial_kernel, DEC_SMEM, smem_set); e != cudaSuccess) return e;
   const int nch = (max_len + DEC_CHUNK - 1) / DEC_CHUNK;
   float* po = scratch;
   float* pml = scratch + (int64_t)B * nq * nch * D;

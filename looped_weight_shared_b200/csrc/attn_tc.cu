@@ -308,12 +308,8 @@ cudaError_t launch_flash_tc(const void* q, const void* K, const void* V, void* o
   if (!map_rows128(&mq, q, (int64_t)B * nq * S, BQ) || !map_rows128(&mk, K, (int64_t)B * nkv * ctx, BKV) ||
       !map_rows128(&mv, V, (int64_t)B * nkv * ctx, BKV))
     return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_limit(flash_tc_kernel, SMEM, smem_set); e != cudaSuccess) return e;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   dim3 grid((unsigned)((S + 2 * BQ - 1) / (2 * BQ)), (unsigned)nq, (unsigned)B);
   flash_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, (bf16*)o, S, nq, nkv, ctx, scale_log2, status_ptr());

@@ -532,12 +532,8 @@ int num_sms() {
 template <Epi MODE>
 cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K, const EpiP& p,
                         cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_limit(gemm_tc_kernel<MODE>, SMEM_BYTES, smem_set); e != cudaSuccess) return e;
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = std::min(tiles, num_sms());
   gemm_tc_kernel<MODE><<<grid, GEMM_THREADS, SMEM_BYTES, st>>>(ma, mb, M, N, K, p, status_ptr());
@@ -570,12 +566,8 @@ cudaError_t launch_gemm_skinny(const void* X, const void* W, int64_t M, int64_t 
   if (!gemm_skinny_supported(M, N, K) || splits < 1) return cudaErrorNotSupported;
   CUtensorMap mw, mx;
   if (!make_map(&mw, W, N, K, BM) || !make_map(&mx, X, M, K, SK_BN)) return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_skinny_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SK_SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_limit(gemm_skinny_kernel, SK_SMEM, smem_set); e != cudaSuccess) return e;
   const int items = (int)((N + BM - 1) / BM) * splits;
   gemm_skinny_kernel<<<std::min(items, num_sms()), THREADS, SK_SMEM, st>>>(mw, mx, (int)M, (int)N, (int)K, splits, P,
                                                                          ldp, status_ptr());

@@ -450,12 +450,8 @@ cudaError_t launch_gla_chunked(const void* q, const void* k, const void* v, cons
   const int64_t rows = (int64_t)B * nh * S;
   if (!map_rows128(&mq, q, rows, CT) || !map_rows128(&mk, k, rows, CT) || !map_rows128(&mv, v, rows, CT))
     return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_limit(gla_tc_kernel, SMEM, smem_set); e != cudaSuccess) return e;
   dim3 grid((unsigned)nh, (unsigned)B);
   gla_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, gl, state, (bf16*)o, S, nh, status_ptr());
   return cudaGetLastError();

@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <string>
 #include <vector>
 
@@ -11,6 +12,21 @@
 #include "common.cuh"
 
 namespace loopk {
+
+// Raise a kernel's dynamic shared-memory limit on the current device, once per
+// device (the setting belongs to that device's context); `done` is the
+// caller's per-kernel bitmask of devices already set.
+template <typename F>
+cudaError_t set_smem_limit(F* kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Output modes of a projection (a GEMM C = A W^T plus what follows it).
 enum class Epi {
