@@ -54,7 +54,7 @@ enum {
 
 enum { LOOP_F32 = 0, LOOP_BF16 = 1 };
 enum { LOOP_TOKENS_TO_LOGITS = 0, LOOP_HIDDEN_TO_HIDDEN = 1 };
-enum { LOOP_ALL_POSITIONS = 1u }; /* loop_prefill flag: logits for every position */
+enum { LOOP_ALL_POSITIONS = 1u }; /* flag of loop_prefill, loop_extend, loop_prefill_ragged: logits for every position */
 enum { LOOP_KIND_LINEAR = 0, LOOP_KIND_FULL = 1 };
 enum { LOOP_REGION_PRELUDE = 0, LOOP_REGION_BLOCK = 1, LOOP_REGION_CODA = 2 };
 
