@@ -86,6 +86,12 @@ def lib():
                 "oracle_seq_len": (i32, [vp, i32]),
                 "oracle_cache_read": (i32, [vp, i32, i32, i32, i32, vp]),
                 "oracle_model_destroy": (None, [vp]),
+                "oracle_attention_sublayer": (i32, [P(Config), vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]),
+                "oracle_gla_sublayer": (i32, [P(Config), vp, vp, vp, vp, vp, vp, vp, i32, i32, vp]),
+                "oracle_ffn_sublayer": (i32, [P(Config), vp, vp, vp, vp, i64, vp]),
+                "oracle_cache_write": (i32, [vp, i32, i32, i32, i32, vp]),
+                "oracle_set_seq_len": (i32, [vp, i32, i32]),
+                "oracle_set_weight": (i32, [vp, i32, vp]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -187,6 +193,55 @@ def mhc_write(s, coef, y):
     return s
 
 
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def attention_sublayer(cfg: Config, wq, wk, wv, wo, xh, start, kcache=None, vcache=None):
+    """The model's full-attention sublayer on caller weights.  xh [B][S][hidden];
+    start[b] is the position of sequence b's first token; the K/V cache slots
+    [B][n_kv][max_ctx][head_dim] are updated in place (zeros if not given).
+    Returns (y [B][S][hidden], kcache, vcache)."""
+    xh = np.ascontiguousarray(xh, dtype=np.float64)
+    B, S, H = xh.shape
+    shape = (cfg.max_batch, cfg.n_kv, cfg.max_ctx, cfg.head_dim)
+    kc = np.zeros(shape, np.float32) if kcache is None else kcache
+    vc = np.zeros(shape, np.float32) if vcache is None else vcache
+    ws = [_f32(w) for w in (wq, wk, wv, wo)]
+    st = np.ascontiguousarray(start, dtype=np.int32)
+    y = np.empty_like(xh)
+    rc = lib().oracle_attention_sublayer(C.byref(cfg), *[_p(w) for w in ws], _p(kc), _p(vc), _p(xh), B, S,
+                                         _p(st), _p(y))
+    if rc != 0:
+        raise ValueError("oracle_attention_sublayer failed")
+    return y, kc, vc
+
+
+def gla_sublayer(cfg: Config, wq, wk, wv, wg, wo, xh, state=None):
+    """The model's gated-linear-attention sublayer on caller weights.  xh
+    [B][S][hidden]; state [B][n_lin][d][d] (zeros if not given) is advanced.
+    Returns (y [B][S][hidden], state)."""
+    xh = np.ascontiguousarray(xh, dtype=np.float64)
+    B, S, H = xh.shape
+    st = np.zeros((B, cfg.n_lin, cfg.lin_dim, cfg.lin_dim)) if state is None else \
+        np.array(state, dtype=np.float64)
+    ws = [_f32(w) for w in (wq, wk, wv, wg, wo)]
+    y = np.empty_like(xh)
+    if lib().oracle_gla_sublayer(C.byref(cfg), *[_p(w) for w in ws], _p(st), _p(xh), B, S, _p(y)) != 0:
+        raise ValueError("oracle_gla_sublayer failed")
+    return y, st
+
+
+def ffn_sublayer(cfg: Config, w_gate, w_up, w_down, xh):
+    """The model's SwiGLU FFN on caller weights; xh [T][hidden] -> y [T][hidden]."""
+    xh = np.ascontiguousarray(xh, dtype=np.float64)
+    ws = [_f32(w) for w in (w_gate, w_up, w_down)]
+    y = np.empty_like(xh)
+    if lib().oracle_ffn_sublayer(C.byref(cfg), *[_p(w) for w in ws], _p(xh), xh.size // xh.shape[-1], _p(y)) != 0:
+        raise ValueError("oracle_ffn_sublayer failed")
+    return y
+
+
 class Model:
     """The oracle's looped decoder with its own KV cache and linear-attention state."""
 
@@ -267,3 +322,27 @@ class Model:
         if lib().oracle_cache_read(self.h, LINEAR, slot, B, 0, _p(out)) != 0:
             raise ValueError("bad state slot")
         return out
+
+    def load_kv(self, slot: int, k: np.ndarray, v: np.ndarray):
+        """Test-only: write K and V [B][n_kv][len][head_dim] into a KV slot."""
+        k, v = _f32(k), _f32(v)
+        B, _, length, _ = k.shape
+        buf = np.ascontiguousarray(np.stack([k, v]))
+        if lib().oracle_cache_write(self.h, FULL, slot, B, length, _p(buf)) != 0:
+            raise ValueError("bad kv slot")
+
+    def load_state(self, slot: int, state: np.ndarray):
+        """Test-only: write the state [B][n_lin][d][d] of a linear slot."""
+        s = _f32(state)
+        if lib().oracle_cache_write(self.h, LINEAR, slot, s.shape[0], 0, _p(s)) != 0:
+            raise ValueError("bad state slot")
+
+    def set_seq_len(self, b: int, length: int):
+        if lib().oracle_set_seq_len(self.h, b, length) != 0:
+            raise ValueError("bad sequence or length")
+
+    def set_weight(self, index: int, values: np.ndarray):
+        """Test-only: replace weight tensor `index` (canonical order)."""
+        x = _f32(values)
+        if x.size != lib().oracle_weight_numel(self.h, index) or lib().oracle_set_weight(self.h, index, _p(x)) != 0:
+            raise ValueError("bad weight index or size")

@@ -293,28 +293,36 @@ void mhc_write_one(double* s, const double* coef, const double* y, int n, int H)
 
 std::vector<double> to_double(const std::vector<float>& v) { return std::vector<double>(v.begin(), v.end()); }
 
-// The full-attention sublayer over B sequences of S new tokens each.
-void full_attention(Model& m, int phys, int slot, const std::vector<double>& xh, int B, int S,
-                    const std::vector<int32_t>& start, std::vector<double>& y) {
-  const oracle_config& c = m.c;
+// Weights of one attention sublayer ([out][in] fp32 values).  wg is the
+// linear-attention gate projection (unused by full attention).
+struct AttnWeights {
+  const float *wq, *wk, *wv, *wg, *wo;
+};
+
+// The full-attention sublayer over B sequences of S new tokens each, the
+// tokens of sequence b at positions start[b] ..: q, k, v projections, RoPE on
+// q and k, K and V appended to the cache slot (K, V: [B][n_kv][max_ctx][hd]),
+// causal softmax attention with kv head = q head / (n_q / n_kv) and scale
+// 1/sqrt(hd), then the output projection into y [T][H].
+void full_attention_core(const oracle_config& c, const AttnWeights& w, float* K, float* V,
+                         const std::vector<double>& xh, int B, int S, const std::vector<int32_t>& start,
+                         std::vector<double>& y) {
   const int64_t T = (int64_t)B * S, H = c.hidden, hd = c.head_dim;
   const int nq = c.n_q, nkv = c.n_kv, grp = nq / nkv;
   std::vector<double> q, k, v;
-  linear(xh, m.w[m.widx_layer(phys, W_Q)].data(), q, T, H, nq * hd);
-  linear(xh, m.w[m.widx_layer(phys, W_K)].data(), k, T, H, nkv * hd);
-  linear(xh, m.w[m.widx_layer(phys, W_V)].data(), v, T, H, nkv * hd);
+  linear(xh, w.wq, q, T, H, nq * hd);
+  linear(xh, w.wk, k, T, H, nkv * hd);
+  linear(xh, w.wv, v, T, H, nkv * hd);
   std::vector<int32_t> pos(T);
   for (int b = 0; b < B; ++b)
     for (int t = 0; t < S; ++t) pos[(int64_t)b * S + t] = start[b] + t;
   rope_rows(q.data(), T, nq, hd, pos.data(), c.rope_base);
   rope_rows(k.data(), T, nkv, hd, pos.data(), c.rope_base);
-  const bool bf = m.bf16();
+  const bool bf = c.dtype == 1;
   for (auto& x : q) x = round_act(x, bf);
   for (auto& x : k) x = round_act(x, bf);
   for (auto& x : v) x = round_act(x, bf);
   // append K, V to this execution's cache slot
-  std::vector<float>& K = m.kc[slot];
-  std::vector<float>& V = m.vc[slot];
   const int64_t L = c.max_ctx;
   for (int b = 0; b < B; ++b)
     for (int t = 0; t < S; ++t)
@@ -331,8 +339,8 @@ void full_attention(Model& m, int phys, int slot, const std::vector<double>& xh,
   for (int b = 0; b < B; ++b)
     for (int h = 0; h < nq; ++h) {
       const int kh = h / grp;
-      const float* Kb = K.data() + ((int64_t)b * nkv + kh) * L * hd;
-      const float* Vb = V.data() + ((int64_t)b * nkv + kh) * L * hd;
+      const float* Kb = K + ((int64_t)b * nkv + kh) * L * hd;
+      const float* Vb = V + ((int64_t)b * nkv + kh) * L * hd;
       std::vector<double> sc;
       for (int t = 0; t < S; ++t) {
         const int p = start[b] + t;
@@ -358,21 +366,22 @@ void full_attention(Model& m, int phys, int slot, const std::vector<double>& xh,
       }
     }
   for (auto& x : o) x = round_act(x, bf);
-  linear(o, m.w[m.widx_layer(phys, W_O)].data(), y, T, nq * hd, H);
+  linear(o, w.wo, y, T, nq * hd, H);
 }
 
-// The gated-linear-attention sublayer: q, k L2-normalised per head, scalar
-// gate g = sigmoid(x W_g) per head; S_t = g_t S_{t-1} + k_t v_t^T, o_t = q_t S_t.
-void linear_attention(Model& m, int phys, int slot, const std::vector<double>& xh, int B, int S,
-                      std::vector<double>& y) {
-  const oracle_config& c = m.c;
+// The gated-linear-attention sublayer: q, k L2-normalised per head (eps
+// inside the square root), scalar gate g = sigmoid(x W_g) per head;
+// S_t = g_t S_{t-1} + k_t v_t^T, o_t = q_t S_t, starting from and leaving the
+// state in `state` [B][n_lin][d][d]; then the output projection into y.
+void linear_attention_core(const oracle_config& c, const AttnWeights& w, double* state,
+                           const std::vector<double>& xh, int B, int S, std::vector<double>& y) {
   const int64_t T = (int64_t)B * S, H = c.hidden, d = c.lin_dim;
   const int nh = c.n_lin;
   std::vector<double> q, k, v, z;
-  linear(xh, m.w[m.widx_layer(phys, W_Q)].data(), q, T, H, nh * d);
-  linear(xh, m.w[m.widx_layer(phys, W_K)].data(), k, T, H, nh * d);
-  linear(xh, m.w[m.widx_layer(phys, W_V)].data(), v, T, H, nh * d);
-  linear(xh, m.w[m.widx_layer(phys, W_G)].data(), z, T, H, nh);
+  linear(xh, w.wq, q, T, H, nh * d);
+  linear(xh, w.wk, k, T, H, nh * d);
+  linear(xh, w.wv, v, T, H, nh * d);
+  linear(xh, w.wg, z, T, H, nh);
   const double eps = c.norm_eps;
   for (int64_t r = 0; r < T * nh; ++r) {
     double sq = 0.0, sk = 0.0;
@@ -386,16 +395,15 @@ void linear_attention(Model& m, int phys, int slot, const std::vector<double>& x
       k[r * d + i] *= ik;
     }
   }
-  const bool bf = m.bf16();
+  const bool bf = c.dtype == 1;
   for (auto& x : q) x = round_act(x, bf);
   for (auto& x : k) x = round_act(x, bf);
   for (auto& x : v) x = round_act(x, bf);
   std::vector<double> o(T * nh * d, 0.0);
-  std::vector<double>& state = m.st[slot];
 #pragma omp parallel for collapse(2) schedule(dynamic)
   for (int b = 0; b < B; ++b)
     for (int h = 0; h < nh; ++h) {
-      double* Sm = state.data() + ((int64_t)b * nh + h) * d * d;
+      double* Sm = state + ((int64_t)b * nh + h) * d * d;
       for (int t = 0; t < S; ++t) {
         const int64_t row = (int64_t)b * S + t;
         const double g = sigmoid(z[row * nh + h]);
@@ -413,18 +421,39 @@ void linear_attention(Model& m, int phys, int slot, const std::vector<double>& x
       }
     }
   for (auto& x : o) x = round_act(x, bf);
-  linear(o, m.w[m.widx_layer(phys, W_O)].data(), y, T, nh * d, H);
+  linear(o, w.wo, y, T, nh * d, H);
 }
 
 // SwiGLU: y = W_down (silu(x W_gate) * (x W_up)).
-void ffn(Model& m, int phys, const std::vector<double>& xh, int64_t T, std::vector<double>& y) {
-  const oracle_config& c = m.c;
+void ffn_core(const oracle_config& c, const float* w_gate, const float* w_up, const float* w_down,
+              const std::vector<double>& xh, int64_t T, std::vector<double>& y) {
   std::vector<double> g, u;
-  linear(xh, m.w[m.widx_layer(phys, W_GATE)].data(), g, T, c.hidden, c.ffn);
-  linear(xh, m.w[m.widx_layer(phys, W_UP)].data(), u, T, c.hidden, c.ffn);
-  const bool bf = m.bf16();
+  linear(xh, w_gate, g, T, c.hidden, c.ffn);
+  linear(xh, w_up, u, T, c.hidden, c.ffn);
+  const bool bf = c.dtype == 1;
   for (int64_t i = 0; i < T * c.ffn; ++i) g[i] = round_act(g[i] * sigmoid(g[i]) * u[i], bf);
-  linear(g, m.w[m.widx_layer(phys, W_DOWN)].data(), y, T, c.ffn, c.hidden);
+  linear(g, w_down, y, T, c.ffn, c.hidden);
+}
+
+AttnWeights layer_weights(const Model& m, int phys) {
+  return {m.w[m.widx_layer(phys, W_Q)].data(), m.w[m.widx_layer(phys, W_K)].data(),
+          m.w[m.widx_layer(phys, W_V)].data(), m.w[m.widx_layer(phys, W_G)].data(),
+          m.w[m.widx_layer(phys, W_O)].data()};
+}
+
+void full_attention(Model& m, int phys, int slot, const std::vector<double>& xh, int B, int S,
+                    const std::vector<int32_t>& start, std::vector<double>& y) {
+  full_attention_core(m.c, layer_weights(m, phys), m.kc[slot].data(), m.vc[slot].data(), xh, B, S, start, y);
+}
+
+void linear_attention(Model& m, int phys, int slot, const std::vector<double>& xh, int B, int S,
+                      std::vector<double>& y) {
+  linear_attention_core(m.c, layer_weights(m, phys), m.st[slot].data(), xh, B, S, y);
+}
+
+void ffn(Model& m, int phys, const std::vector<double>& xh, int64_t T, std::vector<double>& y) {
+  ffn_core(m.c, m.w[m.widx_layer(phys, W_GATE)].data(), m.w[m.widx_layer(phys, W_UP)].data(),
+           m.w[m.widx_layer(phys, W_DOWN)].data(), xh, T, y);
 }
 
 // The forward pass over B sequences of S new tokens starting at start[b].
@@ -637,6 +666,46 @@ void oracle_mhc_write(double* s, const double* coef, const double* y, int32_t n,
   mhc_write_one(s, coef, y, n, H);
 }
 
+// The three sublayers the model runs, on caller arrays (the model calls the
+// same functions with its own weights and cache slots).  xh [B*S][hidden] and
+// y [B*S][hidden] are fp64; weights are fp32 [out][in]; dtype 1 rounds the
+// activations entering matrix products to bf16 as the model does.
+int32_t oracle_attention_sublayer(const oracle_config* c, const float* wq, const float* wk, const float* wv,
+                                  const float* wo, float* kcache, float* vcache, const double* xh, int32_t B,
+                                  int32_t S, const int32_t* start, double* y) {
+  if (!config_ok(c) || B <= 0 || S <= 0 || B > c->max_batch) return -1;
+  for (int b = 0; b < B; ++b)
+    if (start[b] < 0 || start[b] + S > c->max_ctx) return -1;
+  const int64_t T = (int64_t)B * S, H = c->hidden;
+  std::vector<double> x(xh, xh + T * H), out;
+  const AttnWeights w{wq, wk, wv, nullptr, wo};
+  full_attention_core(*c, w, kcache, vcache, x, B, S, std::vector<int32_t>(start, start + B), out);
+  std::memcpy(y, out.data(), sizeof(double) * T * H);
+  return 0;
+}
+
+int32_t oracle_gla_sublayer(const oracle_config* c, const float* wq, const float* wk, const float* wv,
+                            const float* wg, const float* wo, double* state, const double* xh, int32_t B, int32_t S,
+                            double* y) {
+  if (!config_ok(c) || B <= 0 || S <= 0) return -1;
+  const int64_t T = (int64_t)B * S, H = c->hidden;
+  std::vector<double> x(xh, xh + T * H), out;
+  const AttnWeights w{wq, wk, wv, wg, wo};
+  linear_attention_core(*c, w, state, x, B, S, out);
+  std::memcpy(y, out.data(), sizeof(double) * T * H);
+  return 0;
+}
+
+int32_t oracle_ffn_sublayer(const oracle_config* c, const float* w_gate, const float* w_up, const float* w_down,
+                            const double* xh, int64_t T, double* y) {
+  if (!config_ok(c) || T <= 0) return -1;
+  const int64_t H = c->hidden;
+  std::vector<double> x(xh, xh + T * H), out;
+  ffn_core(*c, w_gate, w_up, w_down, x, T, out);
+  std::memcpy(y, out.data(), sizeof(double) * T * H);
+  return 0;
+}
+
 int32_t oracle_num_weights(const oracle_config* c) {
   if (!config_ok(c)) return -1;
   return 2 + W_PER_LAYER * (c->n_prelude + c->n_block + c->n_coda) + 4 * c->n_block;
@@ -756,6 +825,48 @@ int32_t oracle_cache_read(void* mp, int32_t kind, int32_t slot, int32_t B, int32
   if (slot < 0 || slot >= m->n_lin) return -1;
   const int64_t n = (int64_t)B * c.n_lin * c.lin_dim * c.lin_dim;
   for (int64_t i = 0; i < n; ++i) out[i] = (float)m->st[slot][i];
+  return 0;
+}
+
+// Test-only loading of caches: the inverse of oracle_cache_read for sequences
+// 0..B-1 (kind FULL: K then V, [B][n_kv][len][d], positions 0..len-1; kind
+// LINEAR: the state [B][n_lin][dk][dv]).  No arithmetic of the method.
+int32_t oracle_cache_write(void* mp, int32_t kind, int32_t slot, int32_t B, int32_t len, const float* in) {
+  Model* m = (Model*)mp;
+  if (!m || B <= 0 || B > m->c.max_batch) return -1;
+  const oracle_config& c = m->c;
+  if (kind == ORACLE_FULL) {
+    if (slot < 0 || slot >= m->n_full || len < 0 || len > c.max_ctx) return -1;
+    const int64_t hd = c.head_dim, L = c.max_ctx;
+    int64_t o = 0;
+    for (int which = 0; which < 2; ++which) {
+      std::vector<float>& dst = which == 0 ? m->kc[slot] : m->vc[slot];
+      for (int b = 0; b < B; ++b)
+        for (int h = 0; h < c.n_kv; ++h)
+          for (int p = 0; p < len; ++p)
+            for (int i = 0; i < hd; ++i) dst[(((int64_t)b * c.n_kv + h) * L + p) * hd + i] = in[o++];
+    }
+    return 0;
+  }
+  if (slot < 0 || slot >= m->n_lin) return -1;
+  const int64_t n = (int64_t)B * c.n_lin * c.lin_dim * c.lin_dim;
+  for (int64_t i = 0; i < n; ++i) m->st[slot][i] = (double)in[i];
+  return 0;
+}
+
+// Test-only: set the length of sequence b (the position its next token takes).
+int32_t oracle_set_seq_len(void* mp, int32_t b, int32_t len) {
+  Model* m = (Model*)mp;
+  if (!m || b < 0 || b >= m->c.max_batch || len < 0 || len > m->c.max_ctx) return -1;
+  m->seq_len[b] = len;
+  return 0;
+}
+
+// Test-only: replace weight tensor `index` with the caller's values.
+int32_t oracle_set_weight(void* mp, int32_t index, const float* in) {
+  Model* m = (Model*)mp;
+  if (!m || index < 0 || index >= (int)m->w.size()) return -1;
+  std::memcpy(m->w[index].data(), in, sizeof(float) * m->w[index].size());
   return 0;
 }
 

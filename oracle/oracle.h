@@ -72,6 +72,19 @@ void oracle_mhc_site(const double* s, const double* gamma_m, const double* phi, 
                      int32_t n, int32_t H, int32_t iters, double eps, double* coef, double* xhat);
 void oracle_mhc_write(double* s, const double* coef, const double* y, int32_t n, int32_t H);
 
+/* the model's three sublayers on caller arrays (the model runs the same
+ * functions): full attention (K/V cache slot [B][n_kv][max_ctx][head_dim],
+ * appended at start[b] ..), gated linear attention (state [B][n_lin][d][d],
+ * updated in place) and the SwiGLU FFN; xh and y are [B*S][hidden] fp64 */
+int32_t oracle_attention_sublayer(const oracle_config* c, const float* wq, const float* wk, const float* wv,
+                                  const float* wo, float* kcache, float* vcache, const double* xh, int32_t B,
+                                  int32_t S, const int32_t* start, double* y);
+int32_t oracle_gla_sublayer(const oracle_config* c, const float* wq, const float* wk, const float* wv,
+                            const float* wg, const float* wo, double* state, const double* xh, int32_t B, int32_t S,
+                            double* y);
+int32_t oracle_ffn_sublayer(const oracle_config* c, const float* w_gate, const float* w_up, const float* w_down,
+                            const double* xh, int64_t T, double* y);
+
 /* whole model */
 void* oracle_model_create(const oracle_config* c, uint64_t seed, const float* const* weights);
 int32_t oracle_num_weights(const oracle_config* c);
@@ -84,6 +97,11 @@ int32_t oracle_seq_len(void* m, int32_t b);
 /* copies slot `slot` of the KV cache (kind FULL: K then V, [B][n_kv][len][d]) or
  * the GLA state (kind LINEAR: [B][n_lin][dk][dv]) for sequences 0..B-1 */
 int32_t oracle_cache_read(void* m, int32_t kind, int32_t slot, int32_t B, int32_t len, float* out);
+/* test-only: load a cache slot (the layout of oracle_cache_read), set a
+ * sequence's length, replace a weight tensor */
+int32_t oracle_cache_write(void* m, int32_t kind, int32_t slot, int32_t B, int32_t len, const float* in);
+int32_t oracle_set_seq_len(void* m, int32_t b, int32_t len);
+int32_t oracle_set_weight(void* m, int32_t index, const float* in);
 void oracle_model_destroy(void* m);
 
 #ifdef __cplusplus

@@ -337,3 +337,138 @@ def test_mhc_site_coefficients():
     np.testing.assert_allclose(coef[:4], [sig(u[3]), sig(u[8]), 2 * sig(u[1]), 2 * sig(u[10])], rtol=1e-13)
     np.testing.assert_allclose(coef[4:].reshape(1, 2, 2),
                                oracle.sinkhorn_f64(np.array([[[u[2], 0.0], [0.0, 0.0]]]), 20), rtol=1e-13)
+
+
+# --------------------------------------------------------------------------- the model's sublayers
+#
+# The model calls these same oracle functions with its own weights and cache
+# slots, so each hand-computed case below pins the in-model arithmetic.
+
+# Values of the logistic function sigma(x) = 1 / (1 + e^-x), to double precision.
+SIG_1 = 0.7310585786300049
+SIG_2 = 0.8807970779778823
+
+
+def _sub_cfg(**kw):
+    base = dict(n_prelude=0, n_block=4, n_loops=1, n_coda=0, group=4, full_slot=3, hidden=2, ffn=2, vocab=8,
+                n_q=1, n_kv=1, head_dim=2, n_lin=1, lin_dim=2, lin_chunk=64, n_streams=2, sinkhorn_iters=20,
+                rope_base=10000.0, norm_eps=1e-6, dtype=0, io_mode=0, max_batch=1, max_ctx=8)
+    base.update(kw)
+    return oracle.make_config(**base)
+
+
+def test_ffn_sublayer_hand_case():
+    # SwiGLU, y = W_down (silu(x W_gate) * (x W_up)), on x = (1, 2):
+    #   gate = (1, 2), up = (2, 1), silu(z) = z sigma(z)
+    #   a = (1 sigma(1) 2, 2 sigma(2) 1) = (2 sigma(1), 2 sigma(2))
+    #   W_down = [[1, 10], [100, 1000]] -> y = (a0 + 10 a1, 100 a0 + 1000 a1)
+    # Swapping gate and up (or applying silu to up) gives a = (2 sigma(2), 2 sigma(1));
+    # a transposed W_down gives y0 = a0 + 100 a1.
+    cfg = _sub_cfg(hidden=2, ffn=2)
+    a0, a1 = 2 * SIG_1, 2 * SIG_2
+    y = oracle.ffn_sublayer(cfg, np.eye(2), np.array([[0.0, 1.0], [1.0, 0.0]]),
+                            np.array([[1.0, 10.0], [100.0, 1000.0]]), np.array([[1.0, 2.0]]))
+    np.testing.assert_allclose(y, [[a0 + 10 * a1, 100 * a0 + 1000 * a1]], rtol=1e-14)
+
+
+def test_attention_sublayer_gqa_head_map():
+    # 8 query heads over 2 kv heads (group 4, as in the 9B shape), head_dim 2,
+    # hidden 4.  W_q = W_k = 0 makes every score 0, so each head averages the
+    # values of its kv head over the causal prefix; W_v = I gives kv head 0 the
+    # values (x0, x1) and kv head 1 the values (x2, x3).  W_o reads head 1's
+    # output into y0, y1, head 4's first component into y2 and head 7's second
+    # into y3.  With kv head = q head / 4, heads 1 -> kv 0 and heads 4, 7 -> kv 1;
+    # the map q head % 2 would send head 1 to kv 1 and head 4 to kv 0.
+    cfg = _sub_cfg(hidden=4, n_q=8, n_kv=2, head_dim=2, max_ctx=4)
+    wo = np.zeros((4, 16))
+    wo[0, 2], wo[1, 3], wo[2, 8], wo[3, 15] = 1, 1, 1, 1
+    w = (np.zeros((16, 4)), np.zeros((4, 4)), np.eye(4), wo)
+    x = np.array([[[1.0, 2.0, 3.0, 4.0], [5.0, 6.0, 7.0, 8.0]]])
+    y, kc, vc = oracle.attention_sublayer(cfg, *w, x, [0])
+    # t = 0: the one value; t = 1: the mean of two
+    np.testing.assert_allclose(y[0], [[1, 2, 3, 4], [3, 4, 5, 6]], atol=1e-14)
+    np.testing.assert_array_equal(vc[0, :, :2], [[[1, 2], [5, 6]], [[3, 4], [7, 8]]])
+    assert not kc.any()
+    # one more token continuing at position 2 against the cache: mean of three
+    y2, kc, vc = oracle.attention_sublayer(cfg, *w, np.array([[[9.0, 10.0, 11.0, 12.0]]]), [2], kc, vc)
+    np.testing.assert_allclose(y2[0], [[5, 6, 7, 8]], atol=1e-14)
+    np.testing.assert_array_equal(vc[0, :, 2], [[9, 10], [11, 12]])
+
+
+def test_attention_sublayer_scale_and_rope():
+    # One head, head_dim 2, hidden 4.  Token 0: x = (0, 0, 1, 0); token 1:
+    # x = (c, 1, 0, 0) with c = sqrt(2) ln 3.  W_q takes x0 into q's first
+    # component, W_k takes x1 into k's first, W_v maps x -> (x2, x1):
+    #   q(1) = (c, 0), k(0) = (0, 0), k(1) = (1, 0), v(0) = (1, 0), v(1) = (0, 1).
+    # RoPE rotates q(1) and k(1) by the same angle (both at position 1), which
+    # leaves q(1) . k(1) = c; k(0) = 0.  With the scale 1/sqrt(2) the scores of
+    # query 1 are (0, ln 3), so its weights are (1/4, 3/4) and o(1) = (1/4, 3/4).
+    # Without the scale the weights would be (1 + 3^sqrt2)^-1 (1, 3^sqrt2).
+    cfg = _sub_cfg(hidden=4, n_q=1, n_kv=1, head_dim=2, max_ctx=2)
+    c = math.sqrt(2.0) * math.log(3.0)
+    wq = np.array([[1.0, 0, 0, 0], [0, 0, 0, 0]])
+    wk = np.array([[0, 1.0, 0, 0], [0, 0, 0, 0]])
+    wv = np.array([[0, 0, 1.0, 0], [0, 1.0, 0, 0]])
+    wo = np.array([[1.0, 0], [0, 1.0], [0, 0], [0, 0]])
+    x = np.array([[[0, 0, 1.0, 0], [c, 1.0, 0, 0]]])
+    y, kc, _ = oracle.attention_sublayer(cfg, wq, wk, wv, wo, x, [0])
+    np.testing.assert_allclose(y[0], [[1, 0, 0, 0], [0.25, 0.75, 0, 0]], atol=1e-13)
+    # the cached key of position 1 is k(1) rotated by 1 radian (frequency base^0 = 1)
+    np.testing.assert_allclose(kc[0, 0, 1], [math.cos(1.0), math.sin(1.0)], atol=1e-7)
+
+
+# eps = 2^-20 and entries scaled by 2^-10 make every L2 norm exact:
+# |u|^2 = 3 eps gives sqrt(|u|^2 + eps) = 2^-9, |u|^2 = 8 eps gives 3 * 2^-10.
+_EPS = 2.0**-20
+_U = 2.0**-10
+
+
+def test_gla_sublayer_hand_case():
+    # One head, d = 2, hidden 7: x = (q0, q1, k0, k1, v0, v1, z) with identity
+    # projections and the gate z.  q and k are L2-normalised with eps inside
+    # the square root, g = sigmoid(z), S_t = g_t S_{t-1} + k_t v_t^T, o_t = q_t S_t.
+    #   token 0: q = (sqrt3 u, 0) -> q^ = (sqrt3/2, 0); k = (sqrt8 u, 0) -> k^ = (kap, 0),
+    #            kap = sqrt8/3; v = (1, 2); z = 0 -> g = 1/2 (S_0 = 0 anyway)
+    #            S_0 = [[kap, 2 kap], [0, 0]], o_0 = (sqrt3/2)(kap, 2 kap) = (sqrt6/3, 2 sqrt6/3)
+    #   token 1: q = (u, sqrt2 u) -> q^ = (1/2, sqrt2/2); k = (0, sqrt8 u) -> k^ = (0, kap);
+    #            v = (3, 5); z = ln 3 -> g = 3/4
+    #            S_1 = (3/4) S_0 + [[0, 0], [3 kap, 5 kap]] = [[sqrt2/2, sqrt2], [2 sqrt2, 10 sqrt2/3]]
+    #            o_1 = (1/2)(sqrt2/2, sqrt2) + (sqrt2/2)(2 sqrt2, 10 sqrt2/3) = (2 + sqrt2/4, 10/3 + sqrt2/2)
+    # eps outside the root, a log-sigmoid gate, or the gate applied after the
+    # outer product each change these values.
+    cfg = _sub_cfg(hidden=7, n_lin=1, lin_dim=2, norm_eps=_EPS)
+    r2, r3, r6, r8 = math.sqrt(2), math.sqrt(3), math.sqrt(6), math.sqrt(8)
+    x = np.array([[[r3 * _U, 0, r8 * _U, 0, 1, 2, 0], [_U, r2 * _U, 0, r8 * _U, 3, 5, math.log(3.0)]]])
+    eye = np.eye(7)
+    wo = np.zeros((7, 2))
+    wo[0, 0], wo[1, 1] = 1, 1
+    y, st = oracle.gla_sublayer(cfg, eye[0:2], eye[2:4], eye[4:6], eye[6:7], wo, x)
+    np.testing.assert_allclose(y[0, :, :2], [[r6 / 3, 2 * r6 / 3], [2 + r2 / 4, 10 / 3 + r2 / 2]], rtol=1e-13)
+    assert not y[0, :, 2:].any()
+    np.testing.assert_allclose(st[0, 0], [[r2 / 2, r2], [2 * r2, 10 * r2 / 3]], rtol=1e-13)
+
+
+def test_gla_sublayer_equals_recurrence_on_normalised_inputs():
+    # A random case: the sublayer equals the pinned token-by-token recurrence
+    # run on q, k divided by sqrt(|.|^2 + eps) and g = 1 / (1 + e^-z).
+    rng = np.random.default_rng(11)
+    H, nh, d, S = 12, 2, 4, 9
+    cfg = _sub_cfg(hidden=H, n_lin=nh, lin_dim=d, norm_eps=1e-3)
+    wq, wk, wv = (rng.normal(size=(nh * d, H)).astype(np.float32) for _ in range(3))
+    wg = rng.normal(size=(nh, H)).astype(np.float32)
+    wo = rng.normal(size=(H, nh * d)).astype(np.float32)
+    x = rng.normal(size=(1, S, H))
+    s0 = rng.normal(size=(1, nh, d, d))
+    y, st = oracle.gla_sublayer(cfg, wq, wk, wv, wg, wo, x, state=s0)
+    q = (x[0] @ wq.T.astype(np.float64)).reshape(S, nh, d)
+    k = (x[0] @ wk.T.astype(np.float64)).reshape(S, nh, d)
+    v = (x[0] @ wv.T.astype(np.float64)).reshape(S, nh, d)
+    z = x[0] @ wg.T.astype(np.float64)
+    eps = float(np.float32(1e-3))
+    o = np.zeros((S, nh, d))
+    for h in range(nh):
+        qn = q[:, h] / np.sqrt((q[:, h] ** 2).sum(-1, keepdims=True) + eps)
+        kn = k[:, h] / np.sqrt((k[:, h] ** 2).sum(-1, keepdims=True) + eps)
+        o[:, h], sh = oracle.gla_recurrent(qn, kn, v[:, h], 1 / (1 + np.exp(-z[:, h])), state=s0[0, h])
+        np.testing.assert_allclose(st[0, h], sh, atol=1e-12)
+    np.testing.assert_allclose(y[0], o.reshape(S, nh * d) @ wo.T.astype(np.float64), atol=1e-11)
