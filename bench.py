@@ -30,14 +30,14 @@ from seeded import workloads as W  # noqa: E402
 
 DEFAULT_WORKLOAD = "loop9b_prefill_b4_s8192"
 
-# DRAM read + write per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum):
-# - tcgen05 GEMM: mean over the 675 GEMM launches of three 9B prefill steps
-#   (a single-pass ncu launch list of `bench.py --steps 1 --warmup 1`)
+# DRAM read + write per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
+# taken under the small-capture rule; None until taken for the current kernel:
+# - tcgen05 GEMM: per launch of the 9B prefill (see profiles/)
 # - decode attention: 1.085 GB per launch on the probe_decode_b64_ctx4096
 #   workload (64 x 4096 keys), scaled by keys to 32,787
-# Set to None when the kernel changes after the capture.
-GEMM_TRAFFIC_PER_LAUNCH = 3.97e9
+GEMM_TRAFFIC_PER_LAUNCH = None
 DECODE_ATTN_TRAFFIC_PER_LAUNCH = 1.085e9 * 32787 / 4097
+LONG_WORKLOAD = "loop9b_prefill_b1_s262144"
 DATA = "synthetic: seeded SplitMix64 token ids, random-init N(0, 0.02) bf16 weights of the 9B shape"
 
 
@@ -51,7 +51,10 @@ def args_():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=12)
     p.add_argument("--no-decode", action="store_true", help="skip the decode measurement of the default run")
-    p.add_argument("--decode-steps", type=int, default=32)
+    p.add_argument("--decode-steps", type=int, default=None,
+                   help="timed decode steps (default: the decode workload's 128)")
+    p.add_argument("--no-long", action="store_true", help="skip the 262,144-token prefill of the default run")
+    p.add_argument("--long-steps", type=int, default=2)
     return p.parse_args()
 
 
@@ -327,7 +330,8 @@ def run_decode(a, world, local_rank):
     w = W.WORKLOADS["loop9b_decode_b64_ctx32768"]
     m = dict(w["model"])
     B, S, seed = w["batch"], w["seq"], w["seed"]
-    steps, warm = max(a.decode_steps, 1), max(a.warmup, 3)
+    steps = max(a.decode_steps if a.decode_steps is not None else w["decode_steps"], 1)
+    warm = max(a.warmup, 3)
     m.update(max_batch=B, max_ctx=S + warm + 2 * steps + 2)
     g = L.loop_model_create(L.make_config(**m), seed=seed)
     V = m["vocab"]
@@ -370,6 +374,50 @@ def run_decode(a, world, local_rank):
     by = decode_step_bytes(m, B, mid_ctx)
     return {"ms": ms, "value": job_throughput(B, world, ms), "bytes": by, "classes": classes, "clocks": clk.summary(),
             "ctx": mid_ctx, "ms_with_launch_events": ms_timed}
+
+
+def run_long_prefill(a, world, local_rank):
+    """The long-context workload: one 262,144-token prefill of the 9B-shaped
+    model, 1 warm-up step and a.long_steps timed steps, per-class split from
+    CUDA events around every launch (inside the timed region, as for the
+    headline prefill)."""
+    import torch
+    import looped_weight_shared_b200 as L
+
+    dev = torch.device("cuda", local_rank)
+    w = W.WORKLOADS[LONG_WORKLOAD]
+    m = dict(w["model"])
+    B, S, seed = w["batch"], w["seq"], w["seed"]
+    m.update(max_batch=B, max_ctx=S)
+    g = L.loop_model_create(L.make_config(**m), seed=seed)
+    V = m["vocab"]
+    tok = torch.from_numpy(seeded.tokens(seed, B, S, V)).to(dev)
+    out = torch.empty((B, V), device=dev)
+    L.loop_prefill(g, tokens=tok, out=out)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    stream = torch.cuda.current_stream(dev)
+    steps = max(a.long_steps, 1)
+    L.loop_timing_read(g, 0, reset=True)
+    L.loop_set_timing(g, True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        for _ in range(steps):
+            L.loop_prefill(g, tokens=tok, out=out)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    L.loop_set_timing(g, False)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / steps, world, dev)
+    classes = {}
+    for ci, cname in enumerate(L.KERNEL_CLASSES):
+        tms, n, work = L.loop_timing_read(g, ci)
+        classes[cname] = {"ms_per_step": tms / steps, "launches": n, "work": work}
+    status = L.loop_device_status()
+    L.loop_model_destroy(g)
+    return {"ms": ms, "value": job_throughput(B * S, world, ms), "classes": classes, "clocks": clk.summary(),
+            "status": status, "steps": steps, "model": m, "batch": B, "seq": S}
 
 
 # ---------------------------------------------------------------------------- oracle (CPU)
@@ -460,7 +508,8 @@ def main():
     roof = {"bound": "tensor", "kernel": "tcgen05 projection GEMM (all launches in the timed steps)",
             "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak if peak else None,
             "peak_kind": f"{pk_kind} sustained bf16", "traffic": GEMM_TRAFFIC_PER_LAUNCH,
-            "traffic_note": "mean DRAM bytes per GEMM launch (ncu); achieved is over all GEMM launches of the steps"}
+            "traffic_note": "DRAM bytes per GEMM launch (ncu, small-capture rule); achieved is over all GEMM "
+                            "launches of the steps"}
     step_roof = None
     if not decode:
         fl = prefill_step_flops(m, w["batch"], w["seq"])
@@ -498,6 +547,24 @@ def main():
                                  "every launch (ms_per_step_with_launch_events); the headline ms_per_step has none",
             "ms_per_step_with_launch_events": d["ms_with_launch_events"],
             "clocks": d["clocks"]}
+    if a.workload == DEFAULT_WORKLOAD and not a.no_long:
+        lp = run_long_prefill(a, world, local_rank)
+        fl = prefill_step_flops(lp["model"], lp["batch"], lp["seq"])
+        step_tf = fl["total"] / (lp["ms"] / 1e3) / 1e12
+        at = lp["classes"]["attention"]
+        at_tf = at["work"] / (at["ms_per_step"] * lp["steps"]) / 1e9 if at["ms_per_step"] > 0 else 0.0
+        line["long_prefill"] = {
+            "metric": "looped-decoder prefill tokens/s at 9B shape, 262,144-token context", "value": lp["value"],
+            "unit": "tokens/s", "ms_per_step": lp["ms"], "steps": lp["steps"], "warmup": 1,
+            "workload": LONG_WORKLOAD, "batch": lp["batch"], "seq_len": lp["seq"],
+            "step_roofline": {"bound": "tensor", "achieved": step_tf, "peak": peak, "unit": "TFLOP/s",
+                              "frac": step_tf / peak if peak else None, "peak_kind": f"{pk_kind} sustained bf16",
+                              "flops_per_step": fl},
+            "roofline": {"bound": "tensor", "kernel": "tcgen05 causal flash attention (all launches of the steps)",
+                         "achieved": at_tf, "peak": peak, "unit": "TFLOP/s", "frac": at_tf / peak if peak else None,
+                         "peak_kind": f"{pk_kind} sustained bf16", "traffic": None},
+            "kernel_ms_per_step": {k: round(v["ms_per_step"], 3) for k, v in lp["classes"].items()},
+            "device_status": lp["status"], "clocks": lp["clocks"]}
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         c = oracle_sample(a, steps=1)
         line["cpu_baseline"] = {"value": c["value"], "unit": unit, "cores": c["cores"], "kind": "oracle",

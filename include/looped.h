@@ -100,7 +100,14 @@ LOOP_API int32_t loop_schedule(const loop_config* cfg, int32_t* table);
  * Phi [2n + n*n][n*hidden].  Negative status for an invalid configuration. */
 LOOP_API int32_t loop_num_weights(const loop_config* cfg);
 
-/* Create a model.  host_weights == NULL draws every matrix from the seeded
+/* Create a model of the execution configuration *cfg: the loop range
+ * (n_prelude, n_block, n_coda), the pass count n_loops and the mHC settings
+ * that a checkpoint carries and an engine must honour ("How Does
+ * SenseNova-Loop Get More Depth Without More Parameters?", section "How do you
+ * run SenseNova-Loop-9B-Preview?"); the 32-layer, 56-execution shape of the
+ * 9B model is the same page's section "What is the looped decoder in
+ * SenseNova-Loop?".  Invalid configurations give LOOP_EINVAL, valid ones this
+ * library does not run LOOP_EUNSUPPORTED.  host_weights == NULL draws every matrix from the seeded
  * SplitMix64 generator on the device (0.02 * N(0,1), rounded to the model
  * dtype; norm gains 1); otherwise host_weights[i] points to host fp32 values of
  * tensor i in the canonical order above (copied and converted; the caller
@@ -110,7 +117,13 @@ LOOP_API int32_t loop_num_weights(const loop_config* cfg);
 LOOP_API int32_t loop_model_create(const loop_config* cfg, const float* const* host_weights, uint64_t seed,
                           loop_model** out);
 
-/* Prefill B sequences of S tokens from position 0 (resets their caches).
+/* The looped forward pass over a prompt: embedding, prelude layers once, the
+ * shared block n_loops times on its own output with the two mHC streams, the
+ * coda and the tied output head ("How Does SenseNova-Loop Get More Depth
+ * Without More Parameters?", section "What is the looped decoder in
+ * SenseNova-Loop?"; the hybrid 3:1 linear/full attention pattern and its
+ * caches from the section "How does the hybrid attention pattern work?").
+ * Prefill B sequences of S tokens from position 0 (resets their caches).
  * TOKENS_TO_LOGITS: d_tokens int32 [B][S] (each in [0, vocab)); d_out fp32
  *   [B][vocab] with the logits of each sequence's last position, or
  *   [B][S][vocab] when flags has LOOP_ALL_POSITIONS.
@@ -122,7 +135,13 @@ LOOP_API int32_t loop_model_create(const loop_config* cfg, const float* const* h
 LOOP_API int32_t loop_prefill(loop_model* m, const int32_t* d_tokens, const float* d_hidden, int32_t B, int32_t S,
                      float* d_out, uint32_t flags, void* stream);
 
-/* One decode step for sequences 0..B-1: d_tokens int32 [B] is the next token
+/* The same looped forward pass for one new token per sequence, reading and
+ * extending each execution's own KV cache and fixed-size linear-attention state
+ * ("How Does SenseNova-Loop Get More Depth Without More Parameters?", sections
+ * "What is the looped decoder in SenseNova-Loop?" and "How does the hybrid
+ * attention pattern work?": the full-attention cache grows with the context,
+ * the linear-attention state does not; both passes keep their own).
+ * One decode step for sequences 0..B-1: d_tokens int32 [B] is the next token
  * of each sequence, processed at its current length; d_logits fp32 [B][vocab].
  * Appends one KV position per full-attention execution, advances every
  * linear-attention state, then adds 1 to each sequence length.
@@ -198,7 +217,9 @@ LOOP_API int32_t mhc_prologue(const float* d_streams, int64_t T, int32_t H, cons
  * which every GPU that loads the library holds until the process exits.
  * Allocates nothing.  T > 65,536 returns LOOP_ERANGE.  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) with that
- * device current; make that first call before any stream capture.  All calls
+ * device current and keeps it until the process exits; make that first call
+ * before any stream capture, and make no call on a device after a
+ * cudaDeviceReset of it (the kept address is then no longer valid).  All calls
  * on a device share the array and leave their values in it; calls that
  * overlap on the GPU (for instance on two streams) race and must not be
  * issued.  No part of the array needs to start at zero. */
@@ -206,7 +227,11 @@ LOOP_API int32_t mhc_prologue_noalloc(const float* d_streams, int64_t T, int32_t
                                       const float* d_phi, const float* d_gain, int32_t iters, float eps,
                                       float* d_coef, void* d_xhat, int32_t xhat_dtype, void* stream);
 
-/* Release everything the model owns.  Waits for the model's queued work. */
+/* Release everything loop_model_create allocated for the execution
+ * configuration (weights, the per-execution caches of both passes, workspaces;
+ * "How Does SenseNova-Loop Get More Depth Without More Parameters?", section
+ * "How do you run SenseNova-Loop-9B-Preview?").  Waits for the model's queued
+ * work.  NULL is ignored. */
 LOOP_API void loop_model_destroy(loop_model* m);
 
 /* ---- inspection (tests and tools) ---- */
@@ -223,6 +248,20 @@ LOOP_API int32_t loop_cache_read(loop_model* m, int32_t kind, int32_t slot, int3
 /* Copy weight tensor `index` (canonical order, see loop_num_weights) to d_out
  * (device, fp32) in its canonical row-major [out][in] layout. */
 LOOP_API int32_t loop_weight_read(loop_model* m, int32_t index, float* d_out, void* stream);
+
+/* Capture (tests and inspection): while armed, every forward of this model
+ * (prefill, extend, decode) copies, for sequence 0 of the call and heads
+ * [head0, head0 + nheads) of execution `exec`, the inputs and output of its
+ * attention step into caller device buffers (model dtype; NULL skips one):
+ *   linear attention: d_q, d_k, d_v [nheads][S][lin_dim] (q, k L2-normalised),
+ *     d_gate fp32 [nheads][S] (log g), d_o [S][nheads * lin_dim];
+ *   full attention: d_q [nheads][S][head_dim] (after RoPE), d_o as above, and
+ *     d_k, d_v [nk][len][head_dim] for the nk kv heads those query heads read
+ *     (len = the sequence's length after the call), copied from the cache.
+ * S is the number of new tokens of the call.  Up to 8 captures can be armed;
+ * exec < 0 disarms all.  The buffers must stay valid while armed. */
+LOOP_API int32_t loop_capture(loop_model* m, int32_t exec, int32_t head0, int32_t nheads, void* d_q, void* d_k,
+                              void* d_v, float* d_gate, void* d_o);
 
 /* The projection primitive on its own: C[M][N] (row stride ldc, fp32) =
  * A[M][K] W[N][K]^T with A, W bf16 row-major device arrays.  use_tensor_cores

@@ -26,7 +26,7 @@ API = ("loop_num_exec", "loop_schedule", "loop_num_weights", "loop_model_create"
        "loop_decode_step", "mhc_sinkhorn", "loop_model_destroy", "loop_seq_len", "loop_cache_read",
        "loop_weight_read", "loop_device_status", "loop_clear_device_status", "loop_last_error",
        "loop_gemm_bf16", "loop_set_timing", "loop_timing_read", "loop_launch_count", "mhc_prologue",
-       "mhc_prologue_noalloc", "loop_selftest_timeout", "loop_extend", "loop_prefill_ragged")
+       "mhc_prologue_noalloc", "loop_selftest_timeout", "loop_extend", "loop_prefill_ragged", "loop_capture")
 
 
 class loop_config(C.Structure):
@@ -85,6 +85,7 @@ def lib():
             "mhc_prologue": (i32, [vp, C.c_int64, i32, vp, vp, vp, i32, C.c_float, vp, vp, i32, vp, vp]),
             "mhc_prologue_noalloc": (i32, [vp, C.c_int64, i32, vp, vp, vp, i32, C.c_float, vp, vp, i32, vp]),
             "loop_selftest_timeout": (i32, [i32]),
+            "loop_capture": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -200,6 +201,14 @@ def loop_seq_len(model: int, b: int) -> int:
 def loop_cache_read(model: int, kind: int, slot: int, B: int, length: int, out, stream=None) -> None:
     _check("loop_cache_read", lib().loop_cache_read(C.c_void_p(model), kind, slot, B, length, _ptr(out),
                                                     _stream(stream)))
+
+
+def loop_capture(model: int, exec_: int, head0: int = 0, nheads: int = 1, q=None, k=None, v=None, gate=None,
+                 o=None) -> None:
+    """Arm a capture of execution exec_'s attention inputs and output (see
+    include/looped.h); exec_ < 0 disarms every capture."""
+    _check("loop_capture", lib().loop_capture(C.c_void_p(model), exec_, head0, nheads, _ptr(q), _ptr(k), _ptr(v),
+                                              _ptr(gate), _ptr(o)))
 
 
 def loop_weight_read(model: int, index: int, out, stream=None) -> None:

@@ -530,13 +530,13 @@ cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* g
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf,
                                 float* part, cudaStream_t st, int parts, bool fused_read) {
   if (T == 0) return cudaSuccess;
-  if (H % 4 != 0 || mhc_partial_smem(H) > 220 * 1024) return cudaErrorInvalidValue;
+  if (H % 4 != 0 || H > 6144) return cudaErrorInvalidValue;
   if (parts < 2 || parts % 2 != 0 || (2 * H) % (4 * parts) != 0 || H % (2 * H / parts) != 0)
     return cudaErrorInvalidValue;
   const int smem = (int)(mhc_partial_smem(H) * 2 / parts);
-  cudaError_t e = cudaFuncSetAttribute(mhc_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)mhc_partial_smem(H));
-  if (e != cudaSuccess) return e;
+  static std::atomic<uint64_t> smem_set{0};  // the limit for the widest H, raised once per device
+  if (cudaError_t e = set_smem_limit(mhc_partial_kernel, (int)mhc_partial_smem(6144), smem_set); e != cudaSuccess)
+    return e;
   const int64_t per_cta = (int64_t)MHCA_WARPS * MHCA_TOK;
   dim3 ga((unsigned)((T + per_cta - 1) / per_cta), (unsigned)parts);
   mhc_partial_kernel<<<ga, MHCA_THREADS, smem, st>>>(s, T, H, gamma, phi, parts, part);

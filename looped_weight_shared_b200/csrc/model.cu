@@ -62,10 +62,11 @@ bool valid(const loop_config* c) {
 const char* unsupported(const loop_config* c) {
   if (c->n_streams != 2) return "this library runs n_streams == 2";
   if (c->hidden % 4 != 0) return "hidden must be a multiple of 4";
-  if ((size_t)9 * c->hidden * 4 > 220 * 1024) return "hidden must be <= 6144 (mHC prologue keeps Phi in shared memory)";
+  if (c->hidden > 6144) return "hidden must be <= 6144 (mHC prologue keeps Phi in shared memory)";
   if (c->ffn % 128 != 0) return "ffn must be a multiple of 128";
   if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return "head_dim must be 32, 64 or 128";
-  if (c->lin_dim > 256) return "lin_dim must be <= 256";
+  if ((size_t)c->lin_dim * c->lin_dim * 4 + 8 * (size_t)c->lin_dim > 232448)
+    return "lin_dim must be <= 240 (the recurrent kernel keeps the state in shared memory)";
   return nullptr;
 }
 
@@ -492,6 +493,50 @@ cudaError_t linear_attention(Model& m, float* state, int B, int S, cudaStream_t 
   });
 }
 
+// Copy what an armed capture asks for, for sequence 0 of this call (b0 == 0):
+// the attention inputs q (k, v and the log-gates for linear attention; K, V
+// from the cache slot for full attention) and the output o of heads
+// [head0, head0 + nheads), all S positions of this call.
+cudaError_t capture(Model& m, const Capture& cp, bool full, const void* Kc, const void* Vc, int S, cudaStream_t st) {
+  const loop_config& c = m.c;
+  const int64_t es = m.esize;
+  const int64_t nh = full ? c.n_q : c.n_lin, d = full ? c.head_dim : c.lin_dim;
+  const int64_t h0 = cp.head0, n = cp.nheads;
+  // q (and k, v, gates of linear attention): [B][heads][S][d], heads contiguous per sequence
+  if (cp.q)
+    if (cudaError_t e = cudaMemcpyAsync(cp.q, (const char*)m.w.q + h0 * S * d * es, n * S * d * es,
+                                        cudaMemcpyDeviceToDevice, st); e != cudaSuccess) return e;
+  if (full) {
+    // K, V of the kv heads of those query heads, positions 0 .. start + S - 1 of the call
+    const int64_t grp = c.n_q / c.n_kv, kh0 = h0 / grp, nk = (h0 + n - 1) / grp - kh0 + 1;
+    const int64_t len = (m.extending || m.decoding) ? (int64_t)m.seq_len[0] + S : S;
+    for (int64_t j = 0; j < nk; ++j) {
+      const int64_t off = ((kh0 + j) * c.max_ctx) * d * es;
+      if (cp.k)
+        if (cudaError_t e = cudaMemcpyAsync((char*)cp.k + j * len * d * es, (const char*)Kc + off, len * d * es,
+                                            cudaMemcpyDeviceToDevice, st); e != cudaSuccess) return e;
+      if (cp.v)
+        if (cudaError_t e = cudaMemcpyAsync((char*)cp.v + j * len * d * es, (const char*)Vc + off, len * d * es,
+                                            cudaMemcpyDeviceToDevice, st); e != cudaSuccess) return e;
+    }
+  } else {
+    if (cp.k)
+      if (cudaError_t e = cudaMemcpyAsync(cp.k, (const char*)m.w.k + h0 * S * d * es, n * S * d * es,
+                                          cudaMemcpyDeviceToDevice, st); e != cudaSuccess) return e;
+    if (cp.v)
+      if (cudaError_t e = cudaMemcpyAsync(cp.v, (const char*)m.w.v + h0 * S * d * es, n * S * d * es,
+                                          cudaMemcpyDeviceToDevice, st); e != cudaSuccess) return e;
+    if (cp.g)
+      if (cudaError_t e = cudaMemcpyAsync(cp.g, m.w.gl + h0 * S, n * S * 4, cudaMemcpyDeviceToDevice, st);
+          e != cudaSuccess) return e;
+  }
+  // o: [T][heads * d]; rows 0 .. S - 1, the columns of the captured heads
+  if (cp.o)
+    return cudaMemcpy2DAsync(cp.o, n * d * es, (const char*)m.w.o + h0 * d * es, nh * d * es, n * d * es, S,
+                             cudaMemcpyDeviceToDevice, st);
+  return cudaSuccess;
+}
+
 // One forward pass over sequences [b0, b0 + B) with S new tokens each,
 // starting at positions d_start[0..B).  `out` is this group's output.
 int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, int B, int S, const int32_t* d_start,
@@ -560,6 +605,8 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
           qe.heads_q = (int)nq; qe.heads_kv = (int)nkv; qe.hd = (int)hd; qe.cache_ctx = c.max_ctx;
           LOOP_CU(project(m, w.xh, L.w_in, T, L.n_in, H, qe, st));
           LOOP_CU(attention(m, Kc, Vc, B, S, d_start, st));
+          for (const Capture& cp : m.captures)
+            if (cp.exec == e && b0 == 0) LOOP_CU(capture(m, cp, true, Kc, Vc, S, st));
         } else {
           float* state = m.st[slot] + (int64_t)b0 * nl * ld * ld;
           EpiArgs qe;
@@ -568,6 +615,8 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
           qe.S = S; qe.n_lin = (int)nl; qe.hd = (int)ld; qe.eps = c.norm_eps;
           LOOP_CU(project(m, w.xh, L.w_in, T, L.n_in, H, qe, st));
           LOOP_CU(linear_attention(m, state, B, S, st));
+          for (const Capture& cp : m.captures)
+            if (cp.exec == e && b0 == 0) LOOP_CU(capture(m, cp, false, nullptr, nullptr, S, st));
         }
         LOOP_CU(project(m, w.o, L.w_o, T, H, L.n_o_in, out_epi, st));
       } else {
@@ -745,7 +794,7 @@ int32_t mhc_prologue(const float* d_streams, int64_t T, int32_t H, const float* 
                      float* d_scratch, void* stream) {
   if (!d_streams || !d_gamma || !d_phi || !d_gain || !d_coef || !d_xhat || !d_scratch)
     return fail(LOOP_EINVAL, "NULL argument");
-  if (T < 0 || H <= 0 || H % 4 != 0 || mhc_partial_smem(H) > 220 * 1024 || iters < 0 || !(eps >= 0.f))
+  if (T < 0 || H <= 0 || H % 4 != 0 || H > 6144 || iters < 0 || !(eps >= 0.f))
     return fail(LOOP_EINVAL, "T >= 0, H a multiple of 4 and <= 6144, iters >= 0, eps >= 0");
   if (xhat_dtype != LOOP_F32 && xhat_dtype != LOOP_BF16) return fail(LOOP_EINVAL, "bad xhat_dtype");
   LOOP_CU(launch_mhc_prologue(d_streams, T, H, d_gamma, d_phi, d_gain, iters, eps, d_coef, d_xhat,
@@ -828,6 +877,32 @@ int32_t loop_weight_read(loop_model* mp, int32_t index, float* d_out, void* stre
   i -= W_PER_LAYER * m.n_phys;
   const SiteW& s = m.sites[i / 2];
   LOOP_CU(cudaMemcpyAsync(d_out, i % 2 == 0 ? s.gamma : s.phi, rows * cols * 4, cudaMemcpyDeviceToDevice, st));
+  return LOOP_OK;
+}
+
+int32_t loop_capture(loop_model* mp, int32_t exec, int32_t head0, int32_t nheads, void* d_q, void* d_k, void* d_v,
+                     float* d_gate, void* d_o) {
+  if (!mp) return fail(LOOP_EINVAL, "model is NULL");
+  Model& m = mp->m;
+  if (exec < 0) {
+    m.captures.clear();
+    return LOOP_OK;
+  }
+  if (exec >= m.n_exec) return fail(LOOP_EINVAL, "exec out of range");
+  const bool full = m.table[5 * exec + 2] == LOOP_KIND_FULL;
+  const int nh = full ? m.c.n_q : m.c.n_lin;
+  if (head0 < 0 || nheads <= 0 || head0 + nheads > nh) return fail(LOOP_EINVAL, "bad head range");
+  if (m.captures.size() >= 8) return fail(LOOP_ERANGE, "at most 8 captures");
+  Capture cp;
+  cp.exec = exec;
+  cp.head0 = head0;
+  cp.nheads = nheads;
+  cp.q = d_q;
+  cp.k = d_k;
+  cp.v = d_v;
+  cp.g = d_gate;
+  cp.o = d_o;
+  m.captures.push_back(cp);
   return LOOP_OK;
 }
 

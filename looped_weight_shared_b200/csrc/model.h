@@ -96,6 +96,17 @@ struct Work {
   float* dec_attn = nullptr;  // decode attention chunk partials [B][n_q][ctx / 128][130]
 };
 
+// One armed capture of an execution's attention inputs and outputs (test and
+// inspection hook, see loop_capture).
+struct Capture {
+  int exec = -1, head0 = 0, nheads = 0;
+  void* q = nullptr;
+  void* k = nullptr;
+  void* v = nullptr;
+  float* g = nullptr;
+  void* o = nullptr;
+};
+
 struct TimedLaunch {
   int cls;
   double work;
@@ -129,6 +140,7 @@ struct Model {
   bool use_tc = false;          // tcgen05 path for bf16 projections
   bool decoding = false;        // inside loop_decode_step: projections use the decode GEMM
   bool extending = false;       // inside loop_extend: sequences start past 0 (no prefill-only attention)
+  std::vector<Capture> captures;
 };
 
 bool bf16_model(const Model& m);

@@ -30,8 +30,11 @@ std::mutex g_mu;
 float* g_ptr[kMaxDevices] = {};
 
 // The device address of the array on the current device, looked up once per
-// device.  In host code `g_noalloc_scratch` only names a host-side stand-in,
-// so the address must come from cudaGetSymbolAddress.
+// device and kept for the life of the process.  In host code
+// `g_noalloc_scratch` only names a host-side stand-in, so the address must come
+// from cudaGetSymbolAddress.  A cudaDeviceReset on that device invalidates
+// the kept address: callers must not use this entry point after resetting a
+// device it has run on.
 cudaError_t scratch_on_current_device(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -60,7 +63,7 @@ extern "C" int32_t mhc_prologue_noalloc(const float* d_streams, int64_t T, int32
     set_last_error("mhc_prologue_noalloc: NULL argument");
     return LOOP_EINVAL;
   }
-  if (T < 0 || H <= 0 || H % 4 != 0 || mhc_partial_smem(H) > 220 * 1024 || iters < 0 || !(eps >= 0.f)) {
+  if (T < 0 || H <= 0 || H % 4 != 0 || H > 6144 || iters < 0 || !(eps >= 0.f)) {
     set_last_error("mhc_prologue_noalloc: T >= 0, H a multiple of 4 and <= 6144, iters >= 0, eps >= 0");
     return LOOP_EINVAL;
   }

@@ -333,12 +333,14 @@ cudaError_t launch_gla_recurrent(const void* q, const void* k, const void* v, co
                                  bool bf, int B, int S, int nh, int d, cudaStream_t st) {
   if (B == 0 || S == 0) return cudaSuccess;
   const size_t smem = sizeof(float) * ((size_t)d * d + 2 * d);
+  if (smem > 232448) return cudaErrorInvalidValue;
+  static std::atomic<uint64_t> set_bf{0}, set_f{0};  // raised to the per-block maximum once per device
   if (bf) {
-    cudaFuncSetAttribute(gla_recurrent_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (cudaError_t e = set_smem_limit(gla_recurrent_kernel<bf16>, 232448, set_bf); e != cudaSuccess) return e;
     gla_recurrent_kernel<bf16><<<B * nh, d, smem, st>>>((const bf16*)q, (const bf16*)k, (const bf16*)v, gl, state,
                                                         (bf16*)o, S, nh, d);
   } else {
-    cudaFuncSetAttribute(gla_recurrent_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (cudaError_t e = set_smem_limit(gla_recurrent_kernel<float>, 232448, set_f); e != cudaSuccess) return e;
     gla_recurrent_kernel<float><<<B * nh, d, smem, st>>>((const float*)q, (const float*)k, (const float*)v, gl,
                                                          state, (float*)o, S, nh, d);
   }
