@@ -38,6 +38,7 @@ DEFAULT_WORKLOAD = "loop9b_prefill_b4_s8192"
 GEMM_TRAFFIC_PER_LAUNCH = None
 DECODE_ATTN_TRAFFIC_PER_LAUNCH = 1.085e9 * 32787 / 4097
 LONG_WORKLOAD = "loop9b_prefill_b1_s262144"
+EXTEND_K = 8  # tokens per sequence of the timed loop_extend steps
 DATA = "synthetic: seeded SplitMix64 token ids, random-init N(0, 0.02) bf16 weights of the 9B shape"
 
 
@@ -323,6 +324,7 @@ def run_ours(a, rank, world, local_rank):
 
 def run_decode(a, world, local_rank):
     """Decode throughput: 64 sequences after a 32,768-token prefill."""
+    import numpy as np
     import torch
     import looped_weight_shared_b200 as L
 
@@ -332,7 +334,8 @@ def run_decode(a, world, local_rank):
     B, S, seed = w["batch"], w["seq"], w["seed"]
     steps = max(a.decode_steps if a.decode_steps is not None else w["decode_steps"], 1)
     warm = max(a.warmup, 3)
-    m.update(max_batch=B, max_ctx=S + warm + 2 * steps + 2)
+    ek, ewarm, esteps = EXTEND_K, 2, 4  # multi-token append (verify) steps after the decode steps
+    m.update(max_batch=B, max_ctx=S + warm + 2 * steps + ek * (ewarm + esteps) + 2)
     g = L.loop_model_create(L.make_config(**m), seed=seed)
     V = m["vocab"]
     out = torch.empty((B, V), device=dev)
@@ -369,11 +372,27 @@ def run_decode(a, world, local_rank):
     for ci, cname in enumerate(L.KERNEL_CLASSES):
         tms, n, work = L.loop_timing_read(g, ci)
         classes[cname] = {"ms_per_step": tms / steps, "launches": n}
+    # loop_extend: k new tokens per sequence in one pass (the verification step
+    # of multi-token prediction), timed without per-launch events
+    ext = seeded.tokens(seed + 1000, B, ek * (ewarm + esteps), V, stream=seeded.S_DECODE_TOKENS)
+    ext_t = [torch.from_numpy(np.ascontiguousarray(ext[:, i * ek:(i + 1) * ek])).to(dev) for i in range(ewarm + esteps)]
+    for i in range(ewarm):
+        L.loop_extend(g, ext_t[i], out)
+    torch.cuda.synchronize()
+    ectx0 = L.loop_seq_len(g, 0)
+    ev0.record(stream)
+    for i in range(esteps):
+        L.loop_extend(g, ext_t[ewarm + i], out)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ext_ms = max_over_ranks(ev0.elapsed_time(ev1) / esteps, world, dev)
     L.loop_model_destroy(g)
     mid_ctx = ctx0 + steps // 2
     by = decode_step_bytes(m, B, mid_ctx)
     return {"ms": ms, "value": job_throughput(B, world, ms), "bytes": by, "classes": classes, "clocks": clk.summary(),
-            "ctx": mid_ctx, "ms_with_launch_events": ms_timed}
+            "ctx": mid_ctx, "ms_with_launch_events": ms_timed,
+            "extend": {"k": ek, "batch": B, "context": ectx0, "steps": esteps, "warmup": ewarm, "ms_per_step": ext_ms,
+                       "value": job_throughput(B * ek, world, ext_ms), "unit": "tokens/s"}}
 
 
 def run_long_prefill(a, world, local_rank):
@@ -546,6 +565,7 @@ def main():
             "kernel_split_note": "per-class times come from a second run of the same steps with CUDA events around "
                                  "every launch (ms_per_step_with_launch_events); the headline ms_per_step has none",
             "ms_per_step_with_launch_events": d["ms_with_launch_events"],
+            "extend": d["extend"],
             "clocks": d["clocks"]}
     if a.workload == DEFAULT_WORKLOAD and not a.no_long:
         lp = run_long_prefill(a, world, local_rank)

@@ -209,6 +209,7 @@ __global__ void __launch_bounds__(D)
     attn_decode_combine_kernel(const float* __restrict__ po, const float* __restrict__ pml, int nq, int nchunks,
                                bf16* __restrict__ out) {
   const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  griddep_launch_dependents();  // the output projection after this may start streaming its weights
   const int64_t base = ((int64_t)b * nq + h) * nchunks;
   float M = -INFINITY;
   for (int c = 0; c < nchunks; ++c) M = fmaxf(M, pml[(base + c) * 2]);

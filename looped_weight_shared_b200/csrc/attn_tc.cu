@@ -3,22 +3,27 @@
 // Depth Without More Parameters?", section "How does the hybrid attention
 // pattern work?").
 //
-// One CTA computes two 128-query tiles (X = 0, 1: queries q0 .. q0 + 255) of
-// one head against the key tiles of 128 both need, sharing each K/V tile:
+// One CTA computes two 128-query tiles (X = 0, 1: queries q0 .. q0 + 255 of
+// the call, which may continue a sequence: query i at position start + i) of
+// one head against the 64-key tiles both need, sharing each K/V tile:
 //   warp 0      TMA producer: Q of both tiles once, then K and V tiles into a
-//               2-slot ring (128-byte swizzle);
-//   warp 1      allocates TMEM; one lane issues tcgen05.mma, alternating the
-//               tiles so one tile's products run while the other's softmax
-//               does:  S_X = Q_X K_j^T into TMEM, then O_X += P_X V_j with P_X
-//               read from TMEM (it overwrites S_X) and V read in place as an
-//               MN-major B operand;
+//               4-slot ring (128-byte swizzle);
+//   warps 1, 10 one lane each issues the tcgen05.mma of one query tile (warp 1
+//               for tile 0, warp 10 for tile 1, so neither tile's issue order
+//               waits on the other's softmax; warp 1 also allocates TMEM).
+//               Each query tile has two score buffers in TMEM, so the scores
+//               of key tile j + 1 are computed while the softmax of tile j
+//               runs:  S_X(j+1) = Q_X K_{j+1}^T into buffer (j + 1) % 2, then
+//               O_X += P_X(j) V_j with P_X(j) read from TMEM (written over
+//               S_X(j)) and V read in place as an MN-major B operand;
 //   warps 2-5   softmax of tile 0, warps 6-9 softmax of tile 1: thread r owns
-//               query row r of its tile (TMEM lane r), loads its S row, keeps
-//               the running max and sum, writes P (bf16 pairs) back over S,
-//               and rescales its O row in TMEM only when the max grew by more
-//               than 2^8 since the last rescale (the stale max then bounds P
-//               by 256); at the end O / l is stored.
-// TMEM: S_0 (then P_0) at column 0, S_1 at 128, O_0 at 256, O_1 at 384.
+//               query row r of its tile (TMEM lane r), loads its 64 scores,
+//               keeps the running max and sum, writes P (bf16 pairs) back over
+//               S, and rescales its O row in TMEM only when the max grew by
+//               more than 2^8 since the last rescale (the stale max then
+//               bounds P by 256), after the previous P V product is done; at
+//               the end O / l is stored.
+// TMEM: S/P buffers of 64 columns at 64 (2 X + b), O_0 at 256, O_1 at 384.
 // Every mbarrier wait is bounded; the whole warp leaves together before any
 // warp-collective TMEM access.
 
@@ -30,12 +35,14 @@ namespace loopk {
 
 namespace {
 
-constexpr int BQ = 128, BKV = 128, D = 128, NS = 2;
-constexpr int THREADS = 320;             // 2 role warps + 2 softmax warpgroups
+constexpr int BQ = 128, BKV = 64, D = 128, NS = 4;
+constexpr int THREADS = 352;             // producer, MMA tile 0, 2 softmax warpgroups, MMA tile 1
 constexpr int Q_BYTES = BQ * D * 2;      // 32 KB: two boxes [128][64]
-constexpr int KV_TILE = BKV * D * 2;     // 32 KB: two boxes [128][64]
+constexpr int KV_TILE = BKV * D * 2;     // 16 KB: two boxes [64][64]
 constexpr int SMEM = 2 * Q_BYTES + NS * 2 * KV_TILE + 1024 + 256;
+static_assert(SMEM <= 232448, "shared memory per block");
 constexpr int TMEM_COLS = 512;
+constexpr uint32_t T_O = 256;            // O_X at T_O + 128 X
 constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, D, true);
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
@@ -60,15 +67,20 @@ LOOP_DEV float2 exp2_poly2(float2 x) {
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
-// P for 64 keys (S columns 64 hh ..) of one row: p = 2^(s scale - m_ref) as
-// bf16 pairs into pk, their sum added to rs2.  With POLY one pair in three is
-// evaluated on the FMA pipe so the MUFU unit is not the limit.
+LOOP_DEV float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// P for the 64 keys of one row: p = 2^(s scale - m_ref) as bf16 pairs into
+// pk, their sum added to rs2.  With POLY one pair in three is evaluated on the
+// FMA pipe so the MUFU unit is not the limit.
 template <bool POLY>
-LOOP_DEV void softmax_half(const float (&sv)[128], int hh, float2 sc, float2 nm, float (&pk)[32], float2& rs2) {
+LOOP_DEV void softmax_row(const float (&sv)[BKV], float2 sc, float2 nm, float (&pk)[32], float2& rs2) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    const int k = 64 * hh + 2 * i;
-    const float2 xx = ffma2(make_float2(sv[k], sv[k + 1]), sc, nm);
+    const float2 xx = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sc, nm);
     float2 pp;
     if (POLY && (i % 3) == 1)
       pp = exp2_poly2(xx);
@@ -88,7 +100,7 @@ LOOP_DEV uint64_t kmajor_desc(uint32_t base, int rows, int kk) {
 __global__ void __launch_bounds__(THREADS, 1)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, bf16* __restrict__ out, int S, int nq, int nkv,
-                    int64_t ctx, float scale_log2, int* status) {
+                    int64_t ctx, const int32_t* __restrict__ start, float scale_log2, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = smem;                 // tile X at sq + X Q_BYTES
@@ -97,17 +109,20 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + NS;
-  uint64_t* s_full = kv_empty + NS;  // [2] one per query tile
-  uint64_t* p_full = s_full + 2;     // [2]
-  uint64_t* pv_done = p_full + 2;    // [2]
+  uint64_t* s_full = kv_empty + NS;  // [X][buffer]
+  uint64_t* p_full = s_full + 4;     // [X][buffer]
+  uint64_t* pv_done = p_full + 4;    // [X]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
 
   const int npair = (S + 2 * BQ - 1) / (2 * BQ);
   const int q0 = 2 * BQ * (npair - 1 - (int)blockIdx.x);  // longest rows first
   const int h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / (nq / nkv);
+  // query i of the call sits at position p0 + i and sees keys 0 .. p0 + i
+  const int p0 = start ? start[b] : 0;
   // key tiles each query tile needs (0: the second tile is past the end)
-  const int nt[2] = {(min(q0 + BQ, S) - 1) / BKV + 1, q0 + BQ < S ? (min(q0 + 2 * BQ, S) - 1) / BKV + 1 : 0};
+  const int nt[2] = {(p0 + min(q0 + BQ, S) - 1) / BKV + 1,
+                     q0 + BQ < S ? (p0 + min(q0 + 2 * BQ, S) - 1) / BKV + 1 : 0};
   const int ntiles = max(nt[0], nt[1]);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -115,13 +130,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], 2);  // one commit per query tile (the longer tile commits for a missing one)
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], 4);
-      mbar_init(&pv_done[x], 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
     }
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
@@ -154,80 +170,81 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_load_2d(vt, &tv, &kv_full[s], 0, row);
       tma_load_2d(vt + KV_TILE / 2, &tv, &kv_full[s], 64, row);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if ((warp == 1 || warp == 10) && lane == 0) {
+    const int x = warp == 1 ? 0 : 1;  // the query tile this thread issues for
+    const int y = 1 - x;
     const uint32_t q_u = smem_u32(sq), kv_u = smem_u32(skv);
     auto slot = [&](int j) { return kv_u + 2 * (j % NS) * KV_TILE; };
-    // S_X(j) = Q_X K_j^T; P_X of key tile j - 1 must have been consumed
-    auto issue_s = [&](int x, int j) -> bool {
-      if (j >= 1 && !mbar_wait(&pv_done[x], (j - 1) & 1, status, STATUS_WAIT_MMA)) return false;
+    auto sbuf = [&](int j) { return tmem + (uint32_t)(64 * (2 * x + (j & 1))); };
+    // S_X(j) = Q_X K_j^T into buffer j % 2
+    auto issue_s = [&](int j) {
       tc_fence_after();
       const uint32_t kt = slot(j);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        tc_mma_f16(tmem + 128 * x, kmajor_desc(q_u + x * Q_BYTES, BQ, kk), kmajor_desc(kt, BKV, kk), IDESC_S,
+        tc_mma_f16(sbuf(j), kmajor_desc(q_u + x * Q_BYTES, BQ, kk), kmajor_desc(kt, BKV, kk), IDESC_S,
                    kk > 0 ? 1u : 0u);
-      tc_commit(&s_full[x]);
-      return true;
+      tc_commit(&s_full[2 * x + (j & 1)]);
     };
-    // O_X += P_X V_j, P_X read from TMEM
-    auto issue_pv = [&](int x, int j) -> bool {
-      if (!mbar_wait(&p_full[x], j & 1, status, STATUS_WAIT_MMA)) return false;
+    // O_X += P_X(j) V_j, P_X(j) read from TMEM (the first 32 columns of its buffer)
+    auto issue_pv = [&](int j) {
       tc_fence_after();
       const uint32_t vt = slot(j) + KV_TILE;
 #pragma unroll
       for (int kk = 0; kk < BKV / 16; ++kk)
-        tc_mma_f16_ts(tmem + 256 + 128 * x, tmem + 128 * x + 8 * kk,
-                      smem_desc_sw128_lbo(vt + kk * 2048, KV_TILE / 2, 1024), IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+        tc_mma_f16_ts(tmem + T_O + 128 * x, sbuf(j) + 8 * kk, smem_desc_sw128_lbo(vt + kk * 2048, KV_TILE / 2, 1024),
+                      IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
       tc_commit(&pv_done[x]);
-      return true;
     };
     auto kv_ready = [&](int j) { return mbar_wait(&kv_full[j % NS], (j / NS) & 1, status, STATUS_WAIT_MMA); };
-    // order: S_0(0) S_1(0), then per key tile j: PV_0(j) S_0(j+1) PV_1(j)
-    // S_1(j+1), so each tile's next scores start as soon as its own P is used
-    bool ok = mbar_wait(q_full, 0, status, STATUS_WAIT_MMA) && kv_ready(0);
-    for (int x = 0; x < 2 && ok; ++x)
-      if (nt[x] > 0) ok = issue_s(x, 0);
-    for (int j = 0; j < ntiles && ok; ++j) {
-      bool next_loaded = false;
-      for (int x = 0; x < 2 && ok; ++x) {
-        if (j >= nt[x]) continue;
-        ok = issue_pv(x, j);
-        if (ok && j + 1 < nt[x]) {
-          if (!next_loaded) ok = next_loaded = kv_ready(j + 1);
-          if (ok) ok = issue_s(x, j + 1);
-        }
+    bool ok = nt[x] > 0 && mbar_wait(q_full, 0, status, STATUS_WAIT_MMA) && kv_ready(0);
+    if (ok) issue_s(0);
+    for (int j = 0; j < nt[x] && ok; ++j) {
+      if (j + 1 < nt[x]) {
+        // buffer (j + 1) % 2 held P_X(j - 1): its product must be done
+        ok = kv_ready(j + 1) && (j == 0 || mbar_wait(&pv_done[x], (j - 1) & 1, status, STATUS_WAIT_MMA));
+        if (!ok) break;
+        issue_s(j + 1);
       }
-      if (ok) tc_commit(&kv_empty[j % NS]);
+      ok = mbar_wait(&p_full[2 * x + (j & 1)], (j >> 1) & 1, status, STATUS_WAIT_MMA);
+      if (!ok) break;
+      issue_pv(j);
+      // K_j, V_j are free once both tiles' products of key tile j are done;
+      // the longer tile also commits for key tiles the other does not use
+      tc_commit(&kv_empty[j % NS]);
+      if (j >= nt[y]) tc_commit(&kv_empty[j % NS]);
     }
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp < 10) {
     const int x = (warp - 2) >> 2;    // query tile of this warpgroup
     const int quarter = warp & 3;     // TMEM lanes 32 quarter .. (fixed by the warp's rank)
     const int r = 32 * quarter + lane;
-    const int qpos = q0 + BQ * x + r;
+    const int qx0 = q0 + BQ * x;
+    const int qpos = qx0 + r;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    const uint32_t t_s = tmem + 128 * x + lane_off, t_o = tmem + 256 + 128 * x + lane_off;
+    const uint32_t t_o = tmem + T_O + 128 * x + lane_off;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nt[x] && ok; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1, status, STATUS_WAIT_EPILOGUE));
+      const int bi = 2 * x + (j & 1);
+      const uint32_t t_s = tmem + (uint32_t)(64 * bi) + lane_off;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[bi], (j >> 1) & 1, status, STATUS_WAIT_EPILOGUE));
       if (!ok) break;
       tc_fence_after();
       float sv[BKV];
       tmem_ld32(t_s, *reinterpret_cast<float(*)[32]>(sv));
       tmem_ld32(t_s + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
-      tmem_ld32(t_s + 64, *reinterpret_cast<float(*)[32]>(sv + 64));
-      tmem_ld32(t_s + 96, *reinterpret_cast<float(*)[32]>(sv + 96));
       tc_wait_ld();
-      const bool diag = j == nt[x] - 1;  // the key tile on the diagonal (the only one with keys past some rows)
-      if (diag) {
-        const int kbase = j * BKV;
+      const int kbase = j * BKV;
+      const bool masked = kbase + BKV - 1 > p0 + qx0;  // some key of the tile lies past some row's position
+      if (masked) {
 #pragma unroll
         for (int i = 0; i < BKV; ++i)
-          if (kbase + i > qpos) sv[i] = -INFINITY;
+          if (kbase + i > p0 + qpos) sv[i] = -INFINITY;
       }
       float mraw = sv[0];
 #pragma unroll
-      for (int i = 1; i < BKV; ++i) mraw = fmaxf(mraw, sv[i]);
+      for (int i = 1; i + 1 < BKV; i += 2) mraw = max3f(mraw, sv[i], sv[i + 1]);
+      mraw = fmaxf(mraw, sv[BKV - 1]);
       const float mx = mraw * scale_log2;
       float corr = 1.f;
       if (mx > m_ref + RESCALE_THRESHOLD) {
@@ -237,19 +254,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       // p = 2^(s scale - m_ref), two lanes per packed FMA and add
       const float2 sc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
       float2 rs2 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {  // P (bf16 pairs) over S columns 32 hh .., all of S already read
+      {
         float pk[32];
-        if (diag)
-          softmax_half<false>(sv, hh, sc, nm, pk, rs2);
+        if (masked)
+          softmax_row<false>(sv, sc, nm, pk, rs2);
         else
-          softmax_half<true>(sv, hh, sc, nm, pk, rs2);
-        tmem_st32(t_s + 32 * hh, pk);
+          softmax_row<true>(sv, sc, nm, pk, rs2);
+        tmem_st32(t_s, pk);
       }
-      const float rs = rs2.x + rs2.y;
-      l = l * corr + rs;
-      // PV of the last tile finished before S_j was computed, so O is stable
+      l = l * corr + (rs2.x + rs2.y);
+      // rescale O once the product of the previous key tile is done
       if (j >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (j - 1) & 1, status, STATUS_WAIT_EPILOGUE));
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float v[32];
@@ -263,7 +281,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[x]);
+      if (lane == 0) mbar_arrive(&p_full[bi]);
     }
     if (ok && nt[x] > 0) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (nt[x] - 1) & 1, status, STATUS_WAIT_EPILOGUE));
     if (ok && nt[x] > 0) {
@@ -299,10 +317,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 bool flash_tc_supported(int hd, int nq, int nkv) { return hd == D && nq % nkv == 0; }
 
-// q [B][nq][S][128], K/V cache [B][nkv][ctx][128] (positions 0..S-1 valid),
-// o [B*S][nq*128].  All sequences start at position 0.
+// q [B][nq][S][128], K/V cache [B][nkv][ctx][128], o [B*S][nq*128].  The S
+// queries of sequence b sit at positions start[b] .. start[b] + S - 1 (start
+// NULL: from 0) and their keys, positions 0 .. start[b] + S - 1, are in the
+// cache.
 cudaError_t launch_flash_tc(const void* q, const void* K, const void* V, void* o, int B, int S, int nq, int nkv,
-                            int64_t ctx, cudaStream_t st) {
+                            int64_t ctx, const int32_t* start, cudaStream_t st) {
   if (B == 0 || S == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv;
   if (!map_rows128(&mq, q, (int64_t)B * nq * S, BQ) || !map_rows128(&mk, K, (int64_t)B * nkv * ctx, BKV) ||
@@ -312,7 +332,8 @@ cudaError_t launch_flash_tc(const void* q, const void* K, const void* V, void* o
   if (cudaError_t e = set_smem_limit(flash_tc_kernel, SMEM, smem_set); e != cudaSuccess) return e;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   dim3 grid((unsigned)((S + 2 * BQ - 1) / (2 * BQ)), (unsigned)nq, (unsigned)B);
-  flash_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, (bf16*)o, S, nq, nkv, ctx, scale_log2, status_ptr());
+  flash_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, (bf16*)o, S, nq, nkv, ctx, start, scale_log2,
+                                               status_ptr());
   return cudaGetLastError();
 }
 

@@ -77,6 +77,16 @@ LOOP_DEV float log_sigmoidf_(float x) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start before the previous kernel on its
+// stream ends; it must call griddep_wait() before touching anything that
+// kernel writes or reads.  griddep_launch_dependents() lets such a next kernel
+// start.  Both are no-ops without the attribute.
+// ---------------------------------------------------------------------------
+LOOP_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+LOOP_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // shared-memory addresses, mbarriers (every wait is bounded)
 // ---------------------------------------------------------------------------
 LOOP_DEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }

@@ -375,11 +375,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // Output: fp32 partial sums P[split][token][n] (row stride ldp), reduced by
 // the epilogue kernels.
 // ---------------------------------------------------------------------------
-constexpr int SK_BN = 64, SK_STAGES = 6;
-constexpr int SK_A_BYTES = BM * BK * 2;     // weight tile 128 x 64
-constexpr int SK_B_BYTES = SK_BN * BK * 2;  // token tile 64 x 64
+constexpr int SK_BN = 64, SK_BK = 128, SK_STAGES = 4;
+constexpr int SK_A_BYTES = BM * SK_BK * 2;     // weight tile 128 x 128: two 64-column boxes
+constexpr int SK_B_BYTES = SK_BN * SK_BK * 2;  // token tile 64 x 128: two 64-column boxes
 constexpr int SK_STAGE = SK_A_BYTES + SK_B_BYTES;
 constexpr int SK_SMEM = SK_STAGES * SK_STAGE + 1024 + 256;
+static_assert(SK_SMEM <= 232448, "shared memory per block");
 constexpr uint32_t SK_IDESC = idesc_bf16_f32(BM, SK_BN);
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -397,7 +398,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles = (N + BM - 1) / BM, items = tiles * splits;
-  const int kbs = K / BK;
+  const int kbs = K / SK_BK;
   if (threadIdx.x == 0) {
     for (int s = 0; s < SK_STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -417,17 +418,42 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmw);
     prefetch_tmap(&tmx);
-    int stage = 0;
-    uint32_t phase = 0;
+    auto load_w = [&](int stage, int kb, int tile) {
+      tma_load_2d(sw_ + stage * SK_A_BYTES, &tmw, &full[stage], kb * SK_BK, tile * BM);
+      tma_load_2d(sw_ + stage * SK_A_BYTES + SK_A_BYTES / 2, &tmw, &full[stage], kb * SK_BK + 64, tile * BM);
+    };
+    auto load_x = [&](int stage, int kb) {
+      tma_load_2d(sx + stage * SK_B_BYTES, &tmx, &full[stage], kb * SK_BK, 0);
+      tma_load_2d(sx + stage * SK_B_BYTES + SK_B_BYTES / 2, &tmx, &full[stage], kb * SK_BK + 64, 0);
+    };
+    // The weights do not depend on the kernels before this one: the first
+    // ring's worth of weight tiles is requested before waiting for them, the
+    // token tiles of those stages after.
+    int npre = 0, pre_kb[SK_STAGES];
+    for (int it = blockIdx.x; it < items && npre < SK_STAGES; it += gridDim.x) {
+      const int split = it / tiles, tile = it % tiles;
+      const int kb0 = (int)((int64_t)kbs * split / splits), kb1 = (int)((int64_t)kbs * (split + 1) / splits);
+      for (int kb = kb0; kb < kb1 && npre < SK_STAGES; ++kb) {
+        mbar_expect_tx(&full[npre], SK_STAGE);
+        load_w(npre, kb, tile);
+        pre_kb[npre++] = kb;
+      }
+    }
+    griddep_wait();
+    for (int i = 0; i < npre; ++i) load_x(i, pre_kb[i]);
+    int stage = npre % SK_STAGES;
+    uint32_t phase = npre == SK_STAGES ? 1u : 0u;
     bool ok = true;
+    int idx = 0;
     for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
       const int split = it / tiles, tile = it % tiles;
       const int kb0 = (int)((int64_t)kbs * split / splits), kb1 = (int)((int64_t)kbs * (split + 1) / splits);
-      for (int kb = kb0; kb < kb1; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb, ++idx) {
+        if (idx < npre) continue;  // requested above
         if (!mbar_wait(&empty[stage], phase ^ 1, status, STATUS_WAIT_PRODUCER)) { ok = false; break; }
         mbar_expect_tx(&full[stage], SK_STAGE);
-        tma_load_2d(sw_ + stage * SK_A_BYTES, &tmw, &full[stage], kb * BK, tile * BM);
-        tma_load_2d(sx + stage * SK_B_BYTES, &tmx, &full[stage], kb * BK, 0);
+        load_w(stage, kb, tile);
+        load_x(stage, kb);
         if (++stage == SK_STAGES) { stage = 0; phase ^= 1; }
       }
     }
@@ -448,9 +474,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint32_t a0 = smem_u32(sw_ + stage * SK_A_BYTES), b0 = smem_u32(sx + stage * SK_B_BYTES);
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k)
-          tc_mma_f16(d, smem_desc_sw128(a0 + 32 * k, 1024), smem_desc_sw128(b0 + 32 * k, 1024), SK_IDESC,
+        for (int k = 0; k < SK_BK / 16; ++k) {
+          const uint32_t ka = (uint32_t)((k >> 2) * (SK_A_BYTES / 2) + (k & 3) * 32);
+          const uint32_t kx = (uint32_t)((k >> 2) * (SK_B_BYTES / 2) + (k & 3) * 32);
+          tc_mma_f16(d, smem_desc_sw128(a0 + ka, 1024), smem_desc_sw128(b0 + kx, 1024), SK_IDESC,
                      (kb > kb0 || k > 0) ? 1u : 0u);
+        }
         tc_commit(&empty[stage]);
         if (++stage == SK_STAGES) { stage = 0; phase ^= 1; }
       }
@@ -459,6 +488,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp >= 4) {
     const int q = warp & 3;
     int local = 0;
+    griddep_wait();  // the partials may still be read by the kernel before this one
     for (int it = blockIdx.x; it < items; it += gridDim.x, ++local) {
       const int split = it / tiles, tile = it % tiles;
       const int acc = local & 1;
@@ -542,17 +572,17 @@ cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, int M, int
 
 }  // namespace
 
-bool gemm_skinny_supported(int64_t M, int64_t N, int64_t K) { return M >= 1 && M <= SK_BN && K % BK == 0 && N > 0; }
+bool gemm_skinny_supported(int64_t M, int64_t N, int64_t K) { return M >= 1 && M <= SK_BN && K % SK_BK == 0 && N > 0; }
 
 int gemm_skinny_splits(int64_t N, int64_t K) {
   // split-K count minimising the busiest CTA's work: items per CTA times
   // (weight k-blocks per item + ~4 k-block equivalents of fp32 partials
   // written and read back per item)
-  const int64_t tiles = (N + BM - 1) / BM, kbs = K / BK, sms = num_sms();
+  const int64_t tiles = (N + BM - 1) / BM, kbs = K / SK_BK, sms = num_sms();
   int best = 1;
   double best_cost = (double)((tiles + sms - 1) / sms) * (double)kbs;  // one split writes no partials
   for (int s = 2; s <= 16 && s <= kbs; ++s) {
-    const double cost = (double)((tiles * s + sms - 1) / sms) * ((double)kbs / s + 4.0);
+    const double cost = (double)((tiles * s + sms - 1) / sms) * ((double)kbs / s + 2.0);
     if (cost < best_cost * 0.97) {
       best_cost = cost;
       best = s;
@@ -569,9 +599,19 @@ cudaError_t launch_gemm_skinny(const void* X, const void* W, int64_t M, int64_t 
   static std::atomic<uint64_t> smem_set{0};
   if (cudaError_t e = set_smem_limit(gemm_skinny_kernel, SK_SMEM, smem_set); e != cudaSuccess) return e;
   const int items = (int)((N + BM - 1) / BM) * splits;
-  gemm_skinny_kernel<<<std::min(items, num_sms()), THREADS, SK_SMEM, st>>>(mw, mx, (int)M, (int)N, (int)K, splits, P,
-                                                                         ldp, status_ptr());
-  return cudaGetLastError();
+  // programmatic dependent launch: the CTAs start (barriers, TMEM, the first
+  // weight tiles) while the kernel before them finishes
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::min(items, num_sms()));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SK_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_skinny_kernel, mw, mx, (int)M, (int)N, (int)K, splits, P, ldp, status_ptr());
 }
 
 bool gemm_tc_supported(int64_t M, int64_t N, int64_t K, const EpiArgs& e) {

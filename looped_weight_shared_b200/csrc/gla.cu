@@ -39,6 +39,8 @@
 
 #include <cuda.h>
 
+#include <algorithm>
+
 #include "model.h"
 
 namespace loopk {
@@ -82,19 +84,42 @@ LOOP_DEV void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
 
 __global__ void __launch_bounds__(THREADS, 1)
     gla_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                  const __grid_constant__ CUtensorMap tv, const float* __restrict__ gl, float* __restrict__ state,
-                  bf16* __restrict__ out, int S, int nh, int* status) {
+                  const __grid_constant__ CUtensorMap tv, const float* __restrict__ gl,
+                  const float* __restrict__ init_state, float* __restrict__ seg_states,
+                  float* __restrict__ final_state, bf16* __restrict__ out, int S, int nh, int nseg, int seg_tiles,
+                  int pass, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* b2s = reinterpret_cast<float*>(smem + OFF_B2);  // [NB2][CT] running log2 gates
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + NBARS);
 
-  const int h = blockIdx.x, b = blockIdx.y;
+  const int h = blockIdx.x, b = blockIdx.y, seg = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nch = (S + CT - 1) / CT;
-  const int row0 = (b * nh + h) * S;  // first row of this head in the [B nh S][128] views
+  // this CTA's segment: tokens t0 .. t0 + Sl - 1 of the sequence, walked as a
+  // sequence of its own from the segment's start state
+  const int t0 = seg * seg_tiles * CT;
+  const int Sl = min(S - t0, seg_tiles * CT);
+  const int nch = (Sl + CT - 1) / CT;
+  const int row0 = (b * nh + h) * S + t0;  // first row of this segment in the [B nh S][128] views
   const int64_t bh = (int64_t)b * nh + h;
+  // start state (NULL: zero) and where the end state goes (NULL: nowhere).
+  // One segment: init_state to final_state.  Several (seg_states holds nseg
+  // states per head): pass 1 runs segments 0 .. nseg - 2 from zero and leaves
+  // segment p's local end state in slot p + 1; gla_scan_kernel turns slot p
+  // into the true start state of segment p; pass 2 runs every segment from its
+  // slot and the last one writes final_state.
+  const float* s_in = nullptr;
+  float* s_out = nullptr;
+  if (nseg == 1) {
+    s_in = init_state + bh * DK * 128;
+    s_out = final_state + bh * DK * 128;
+  } else if (pass == 1) {
+    s_out = seg_states + (bh * nseg + seg + 1) * (int64_t)DK * 128;
+  } else {
+    s_in = seg_states + (bh * nseg + seg) * (int64_t)DK * 128;
+    if (seg == nseg - 1) s_out = final_state + bh * DK * 128;
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBARS; ++i) mbar_init(&bar[i], i >= B_SR ? 8u : 1u);
@@ -183,7 +208,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int cb = 64 * (ew >> 2);    // this warp's column half
     const int r = 32 * quarter + lane;  // the row this thread owns: token t, key s or state row
     const uint32_t lo_lane = (uint32_t)(32 * quarter) << 16;
-    const float* glh = gl + bh * S;
+    const float* glh = gl + bh * S + t0;
     bool ok = true;
 
     // running sums of the log gates of tile j, in log2 units (0 past the end)
@@ -191,7 +216,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ew != 0) return true;
       if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bar[B_SR], (j - 1) & 1, status, STATUS_WAIT_EPILOGUE)))
         return false;  // every warp has read the gate buffer this one reuses
-      const int c0 = j * CT, valid = min(CT, S - c0);
+      const int c0 = j * CT, valid = min(CT, Sl - c0);
       float x[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) x[i] = 4 * lane + i < valid ? glh[c0 + 4 * lane + i] : 0.f;
@@ -221,7 +246,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
       }
       const float dl = ex2(b2s[(j % NB2) * CT + CT - 1]);
-      const float* src = state + (bh * DK + r) * 128;
+      const float* src = s_in ? s_in + r * 128 : nullptr;
 #pragma unroll 1
       for (int hh = 0; hh < 2; ++hh) {
         const int col = cb + 32 * hh;
@@ -229,7 +254,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (j == 0) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float4 v = reinterpret_cast<const float4*>(src + col)[i];
+            const float4 v = src ? reinterpret_cast<const float4*>(src + col)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
             s[4 * i] = v.x;
             s[4 * i + 1] = v.y;
             s[4 * i + 2] = v.z;
@@ -263,9 +288,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
     // the final state of the sequence back to global memory
     auto state_out = [&](int last) -> bool {
+      if (!s_out) return true;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_DS], last & 1, status, STATUS_WAIT_EPILOGUE))) return false;
       tc_fence_after();
-      float* dst = state + (bh * DK + r) * 128;
+      float* dst = s_out + r * 128;
 #pragma unroll 1
       for (int hh = 0; hh < 2; ++hh) {
         const int col = cb + 32 * hh;
@@ -282,7 +308,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto vhat = [&](int j) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_VF], j & 1, status, STATUS_WAIT_EPILOGUE))) return false;
       const float* bb = b2s + (j % NB2) * CT;
-      const int valid = min(CT, S - j * CT);
+      const int valid = min(CT, Sl - j * CT);
       const float w = r < valid ? ex2(bb[CT - 1] - bb[r]) : 0.f;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
@@ -308,7 +334,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_PF], j & 1, status, STATUS_WAIT_EPILOGUE))) return false;
       tc_fence_after();
       const float* bb = b2s + (j % NB2) * CT;
-      const int valid = min(CT, S - j * CT);
+      const int valid = min(CT, Sl - j * CT);
       const float bt = bb[r];
       const bool row_ok = r < valid;
 #pragma unroll 1
@@ -338,9 +364,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto output = [&](int c) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_OF], c & 1, status, STATUS_WAIT_EPILOGUE))) return false;
       tc_fence_after();
-      const int c0 = c * CT, valid = min(CT, S - c0);
+      const int c0 = c * CT, valid = min(CT, Sl - c0);
       const float et = ex2(b2s[(c % NB2) * CT + r]);
-      bf16* dst = out + ((int64_t)b * S + c0 + r) * ((int64_t)nh * 128) + h * 128;
+      bf16* dst = out + ((int64_t)b * S + t0 + c0 + r) * ((int64_t)nh * 128) + h * 128;
 #pragma unroll 1
       for (int hh = 0; hh < 2; ++hh) {
         const int col = cb + 32 * hh;
@@ -383,6 +409,52 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
+// The chaining step between the two passes of a segmented prefill, one CTA
+// per (sequence, head): slot 0 = the initial state, then for p = 1 .. nseg - 1
+//   slot p = G_{p-1} slot (p - 1) + slot p,  G_{p-1} = exp(sum of log g over
+// segment p - 1), where slot p held segment p - 1's local end state (its
+// state from zero).  This is the recurrence S_t = g_t S_{t-1} + k_t v_t^T
+// taken a segment at a time.  The gate sums are accumulated in fp64.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    gla_scan_kernel(const float* __restrict__ gl, const float* __restrict__ init_state,
+                    float* __restrict__ seg_states, int S, int nseg, int seg_tokens) {
+  __shared__ double red[8];
+  const int64_t bh = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  float* base = seg_states + bh * nseg * (int64_t)DK * 128;
+  const float* init = init_state ? init_state + bh * DK * 128 : nullptr;
+  float cur[64];  // this thread's 64 state entries of the current slot
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const int e = i * 256 + tid;
+    cur[i] = init ? init[e] : 0.f;
+    base[e] = cur[i];
+  }
+  for (int p = 1; p < nseg; ++p) {
+    const float* g = gl + bh * S + (int64_t)(p - 1) * seg_tokens;
+    double acc = 0.0;
+    for (int t = tid; t < seg_tokens; t += 256) acc += (double)g[t];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) red[wid] = acc;
+    __syncthreads();
+    double tot = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    __syncthreads();
+    const float decay = (float)exp(tot);
+    float* slot = base + (int64_t)p * DK * 128;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      const int e = i * 256 + tid;
+      cur[i] = fmaf(decay, cur[i], slot[e]);
+      slot[e] = cur[i];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // One decode step of gated linear attention (d = 128): S = g S + k v^T,
 // o = q S.  CTA (32-column slice of S, head, sequence), 256 threads: thread
 // (row group rg = tid / 32, column c = tid % 32) updates rows 16 rg .. 16 rg + 15
@@ -393,6 +465,7 @@ __global__ void __launch_bounds__(256)
     gla_decode_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
                       const float* __restrict__ gl, float* __restrict__ state, bf16* __restrict__ out, int nh) {
   __shared__ float qs[DK], ks[DK], red[8][32];
+  griddep_launch_dependents();  // the output projection after this may start streaming its weights
   const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, rg = tid >> 5, c = tid & 31;
   const int64_t bh = (int64_t)b * nh + h;
@@ -443,8 +516,11 @@ cudaError_t launch_gla_decode(const void* q, const void* k, const void* v, const
 
 // q, k, v [B][nh][S][128] bf16; gl [B][nh][S] log-gates; state [B][nh][128][128]
 // fp32 (read, then replaced by the final state); o [B*S][nh*128] bf16.
+// seg_scratch (may be NULL) holds scratch_floats floats; with room, a batch
+// with fewer (sequence, head) pairs than SMs is cut into segments of whole
+// tiles so the segments run in parallel (two passes and a scan).
 cudaError_t launch_gla_chunked(const void* q, const void* k, const void* v, const float* gl, float* state, void* o,
-                               int B, int S, int nh, cudaStream_t st) {
+                               int B, int S, int nh, float* seg_scratch, int64_t scratch_floats, cudaStream_t st) {
   if (B == 0 || S == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv;
   const int64_t rows = (int64_t)B * nh * S;
@@ -452,8 +528,28 @@ cudaError_t launch_gla_chunked(const void* q, const void* k, const void* v, cons
     return cudaErrorInvalidValue;
   static std::atomic<uint64_t> smem_set{0};
   if (cudaError_t e = set_smem_limit(gla_tc_kernel, SMEM, smem_set); e != cudaSuccess) return e;
-  dim3 grid((unsigned)nh, (unsigned)B);
-  gla_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, gl, state, (bf16*)o, S, nh, status_ptr());
+  const int nch = (S + CT - 1) / CT;
+  int nseg = 1;
+  if (seg_scratch) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int pairs = B * nh;
+    nseg = std::max(1, std::min(sms / std::max(pairs, 1), nch / 8));  // at least 8 tiles a segment
+    while (nseg > 1 && (int64_t)pairs * nseg * DK * 128 > scratch_floats) --nseg;
+  }
+  const int seg_tiles = (nch + nseg - 1) / nseg;
+  nseg = (nch + seg_tiles - 1) / seg_tiles;  // no empty segment
+  int* status = status_ptr();
+  if (nseg == 1) {
+    gla_tc_kernel<<<dim3((unsigned)nh, (unsigned)B, 1), THREADS, SMEM, st>>>(
+        mq, mk, mv, gl, state, nullptr, state, (bf16*)o, S, nh, 1, seg_tiles, 2, status);
+    return cudaGetLastError();
+  }
+  gla_tc_kernel<<<dim3((unsigned)nh, (unsigned)B, (unsigned)(nseg - 1)), THREADS, SMEM, st>>>(
+      mq, mk, mv, gl, nullptr, seg_scratch, nullptr, (bf16*)o, S, nh, nseg, seg_tiles, 1, status);
+  gla_scan_kernel<<<(unsigned)(B * nh), 256, 0, st>>>(gl, state, seg_scratch, S, nseg, seg_tiles * CT);
+  gla_tc_kernel<<<dim3((unsigned)nh, (unsigned)B, (unsigned)nseg), THREADS, SMEM, st>>>(
+      mq, mk, mv, gl, nullptr, seg_scratch, state, (bf16*)o, S, nh, nseg, seg_tiles, 2, status);
   return cudaGetLastError();
 }
 

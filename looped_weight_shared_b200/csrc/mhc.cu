@@ -110,6 +110,7 @@ cudaError_t launch_embed(const int32_t* tok, const void* E, bool bf, int64_t T, 
 template <typename T>
 __global__ void rmsnorm_kernel(const float* x, int H, int64_t step, int64_t off, const float* gain, float eps, T* y) {
   __shared__ float red[32];
+  griddep_launch_dependents();  // a decode GEMM after this may start streaming its weights
   const int64_t r = blockIdx.x;
   const float* xr = x + (r * step + off) * H;
   float ss = 0.f;
@@ -427,6 +428,7 @@ __global__ void __launch_bounds__(256)
                      float* __restrict__ coef, T* __restrict__ xh) {
   constexpr int H = 1024 * NK, H4 = H / 4, D = 2 * H;
   __shared__ float red[8][9];
+  griddep_launch_dependents();  // the decode GEMM after this may start streaming its weights
   __shared__ float cf[2];
   __shared__ float red2[8];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

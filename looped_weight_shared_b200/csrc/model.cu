@@ -324,6 +324,10 @@ int32_t create_impl(const loop_config* cfg, const float* const* hw, uint64_t see
     w.cpart_floats = 32 * 64 * maxn;
     LOOP_ALLOC(w.cpart, float*, w.cpart_floats * 4);
   }
+  if (bf && gla_chunk_supported((int)ld)) {  // one state per SM: the most a segmented prefill uses
+    w.gla_seg_floats = 160 * ld * ld;
+    LOOP_ALLOC(w.gla_seg, float*, w.gla_seg_floats * 4);
+  }
   if (bf && decode_attention_supported((int)hd, (int)nq, (int)nkv))
     LOOP_ALLOC(w.dec_attn, float*, decode_attention_scratch_floats((int)Bm, (int)nq, ctx) * 4);
   LOOP_ALLOC(w.q, void*, T * qw * es);
@@ -443,9 +447,10 @@ cudaError_t project(Model& m, const void* A, const void* W, int64_t M, int64_t N
 cudaError_t attention(Model& m, const void* Kc, const void* Vc, int B, int S, const int32_t* d_start, cudaStream_t st) {
   const loop_config& c = m.c;
   const bool bf = bf16_model(m);
-  // algorithmic FLOPs: QK^T and PV over the causal keys, assuming the
-  // sequences start at position 0 for a prefill (S > 1) or at S - 1 keys back
-  const double pairs = (double)B * S * (S + 1) / 2.0;
+  // algorithmic FLOPs: QK^T and PV over the causal keys of every query
+  double pairs = (double)B * S * (S + 1) / 2.0;
+  if (m.extending)
+    for (int b = 0; b < B; ++b) pairs += (double)S * m.seq_len[b];
   const double flops = 4.0 * pairs * c.head_dim * c.n_q;
   if (bf && S == 1 && m.w.dec_attn && decode_attention_supported(c.head_dim, c.n_q, c.n_kv)) {
     // one new token per sequence: its key position is seq_len[b]; the keys
@@ -462,9 +467,10 @@ cudaError_t attention(Model& m, const void* Kc, const void* Vc, int B, int S, co
                                      m.w.dec_attn, st);
     });
   }
-  if (bf && S > 1 && !m.extending && flash_tc_supported(c.head_dim, c.n_q, c.n_kv))  // a prefill: every sequence starts at 0
+  if (bf && S > 1 && flash_tc_supported(c.head_dim, c.n_q, c.n_kv))  // prefill from 0, or extend from seq_len
     return timed(m, LOOP_K_ATTENTION, flops, 1, st, [&] {
-      return launch_flash_tc(m.w.q, Kc, Vc, m.w.o, B, S, c.n_q, c.n_kv, c.max_ctx, st);
+      return launch_flash_tc(m.w.q, Kc, Vc, m.w.o, B, S, c.n_q, c.n_kv, c.max_ctx, m.extending ? d_start : nullptr,
+                             st);
     });
   return timed(m, LOOP_K_ATTENTION, flops, 1, st, [&] {
     return launch_attention_simple(m.w.q, Kc, Vc, m.w.o, bf, B, S, c.n_q, c.n_kv, c.head_dim, c.max_ctx, d_start, st);
@@ -480,7 +486,8 @@ cudaError_t linear_attention(Model& m, float* state, int B, int S, cudaStream_t 
     // chunked form: Q K^T, (.)V, Q S and K^T V per chunk of 64 tokens
     const double flops = 4.0 * (double)B * S * c.n_lin * d * (64.0 + d);
     return timed(m, LOOP_K_LINEAR_ATTENTION, flops, 1, st, [&] {
-      return launch_gla_chunked(m.w.q, m.w.k, m.w.v, m.w.gl, state, m.w.o, B, S, c.n_lin, st);
+      return launch_gla_chunked(m.w.q, m.w.k, m.w.v, m.w.gl, state, m.w.o, B, S, c.n_lin, m.w.gla_seg,
+                                m.w.gla_seg_floats, st);
     });
   }
   const double flops = 4.0 * (double)B * S * c.n_lin * d * d;

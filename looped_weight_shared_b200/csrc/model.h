@@ -94,6 +94,8 @@ struct Work {
   float* cpart = nullptr;     // split-K partial sums of the decode GEMM [32][64][max N]
   int64_t cpart_floats = 0;
   float* dec_attn = nullptr;  // decode attention chunk partials [B][n_q][ctx / 128][130]
+  float* gla_seg = nullptr;   // segment states of a segmented linear-attention prefill
+  int64_t gla_seg_floats = 0;
 };
 
 // One armed capture of an execution's attention inputs and outputs (test and
@@ -139,7 +141,7 @@ struct Model {
   std::vector<void*> allocs;
   bool use_tc = false;          // tcgen05 path for bf16 projections
   bool decoding = false;        // inside loop_decode_step: projections use the decode GEMM
-  bool extending = false;       // inside loop_extend: sequences start past 0 (no prefill-only attention)
+  bool extending = false;       // inside loop_extend: sequences start past 0 (attention starts at seq_len)
   std::vector<Capture> captures;
 };
 
@@ -197,10 +199,11 @@ cudaError_t launch_set_len(int32_t* seq_len, int B, int S, cudaStream_t st);
 cudaError_t launch_weight_to_f32(const void* src, bool bf16, int64_t rows, int64_t cols, int64_t src_row0,
                                  float* dst, cudaStream_t st);
 
-// flash attention for prefill on tcgen05 (bf16, head_dim 128, all sequences from position 0)
+// flash attention on tcgen05 (bf16, head_dim 128) for S queries per sequence
+// at positions start[b] .. (start NULL: from 0)
 bool flash_tc_supported(int hd, int nq, int nkv);
 cudaError_t launch_flash_tc(const void* q, const void* K, const void* V, void* o, int B, int S, int nq, int nkv,
-                            int64_t ctx, cudaStream_t st);
+                            int64_t ctx, const int32_t* start, cudaStream_t st);
 
 // decode attention (flash-decoding over 128-key chunks; bf16, head_dim 128, group 4)
 bool decode_attention_supported(int hd, int nq, int nkv);
@@ -210,8 +213,10 @@ cudaError_t launch_attention_decode(const void* q, const void* K, const void* V,
 
 // chunked gated linear attention for prefill (bf16, d = 128)
 bool gla_chunk_supported(int d);
+// seg_scratch (may be NULL, scratch_floats floats) lets a small batch run as
+// parallel segments of each sequence
 cudaError_t launch_gla_chunked(const void* q, const void* k, const void* v, const float* gl, float* state, void* o,
-                               int B, int S, int nh, cudaStream_t st);
+                               int B, int S, int nh, float* seg_scratch, int64_t scratch_floats, cudaStream_t st);
 
 // one decode step of gated linear attention (bf16, d = 128)
 cudaError_t launch_gla_decode(const void* q, const void* k, const void* v, const float* gl, float* state, void* o,

@@ -107,6 +107,7 @@ __global__ void epi_mhc_kernel(CView C, int64_t M, int64_t N, float* s, const fl
 
 template <typename T>
 __global__ void epi_swiglu_kernel(CView C, int64_t M, int64_t F, T* a) {
+  griddep_launch_dependents();  // the down projection after this may start streaming its weights
   const int64_t n = M * F;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / F, f = i % F;

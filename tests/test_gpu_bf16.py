@@ -238,3 +238,30 @@ def test_mid_bf16_mixed_length_decode():
         assert L.loop_device_status() == 0
     finally:
         L.loop_model_destroy(g)
+
+
+def test_mid_bf16_extend_after_ragged_prefill():
+    """loop_extend of k = 8 tokens on sequences of different lengths: the
+    tensor-core flash kernel with a different start position per sequence
+    (keys before the new positions, the causal block among them), each
+    sequence against its own oracle's decode steps."""
+    lens, k = [1100, 77, 530], 8
+    m = dict(W.model_config("tiny_fp32", **MID4), max_batch=3, max_ctx=1120)
+    g = L.loop_model_create(L.make_config(**m), seed=12)
+    try:
+        seqs = [seeded.tokens(70 + i, 1, n, m["vocab"])[0] for i, n in enumerate(lens)]
+        os_ = [oracle.Model(oracle.make_config(**m), seed=12) for _ in lens]
+        for o, s in zip(os_, seqs):
+            o.prefill(s[None, :])
+        out = torch.empty((3, m["vocab"]), device="cuda")
+        L.loop_prefill_ragged(g, torch.from_numpy(np.concatenate(seqs)).cuda(), lens, out)
+        ext = seeded.tokens(71, 3, k, m["vocab"], stream=seeded.S_DECODE_TOKENS)
+        got = torch.empty((3, k, m["vocab"]), device="cuda")
+        L.loop_extend(g, torch.from_numpy(ext).cuda(), got, flags=L.LOOP_ALL_POSITIONS)
+        torch.cuda.synchronize()
+        ref = np.stack([np.concatenate([o.decode_step(ext[i, t:t + 1]) for t in range(k)]) for i, o in enumerate(os_)])
+        check(got.cpu().numpy(), ref)
+        assert [L.loop_seq_len(g, i) for i in range(3)] == [n + k for n in lens]
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
