@@ -100,7 +100,7 @@ LOOP_DEV uint64_t kmajor_desc(uint32_t base, int rows, int kk) {
 __global__ void __launch_bounds__(THREADS, 1)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, bf16* __restrict__ out, int S, int nq, int nkv,
-                    int64_t ctx, const int32_t* __restrict__ start, float scale_log2, int* status) {
+                    int64_t ctx, const int32_t* __restrict__ start, int packed, float scale_log2, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = smem;                 // tile X at sq + X Q_BYTES
@@ -114,15 +114,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* pv_done = p_full + 4;    // [X]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
 
+  // Unpacked: CTA (query-tile pair, query head, sequence).  Packed (a few new
+  // tokens per sequence, grp * S <= 128): CTA (kv head, sequence) whose one
+  // tile holds the S queries of each of the grp query heads sharing that kv
+  // head, row r = (head kvh * grp + r / S, query r % S): the heads' q rows are
+  // adjacent in q, so one box loads them, and K/V are read once per kv head.
+  const int grp = nq / nkv;
   const int npair = (S + 2 * BQ - 1) / (2 * BQ);
-  const int q0 = 2 * BQ * (npair - 1 - (int)blockIdx.x);  // longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int kvh = h / (nq / nkv);
+  const int q0 = packed ? 0 : 2 * BQ * (npair - 1 - (int)blockIdx.x);  // longest rows first
+  const int b = blockIdx.z;
+  const int kvh = packed ? (int)blockIdx.y : (int)blockIdx.y / grp;
+  const int h = packed ? kvh * grp : (int)blockIdx.y;  // the (first) query head
   // query i of the call sits at position p0 + i and sees keys 0 .. p0 + i
   const int p0 = start ? start[b] : 0;
   // key tiles each query tile needs (0: the second tile is past the end)
   const int nt[2] = {(p0 + min(q0 + BQ, S) - 1) / BKV + 1,
-                     q0 + BQ < S ? (p0 + min(q0 + 2 * BQ, S) - 1) / BKV + 1 : 0};
+                     !packed && q0 + BQ < S ? (p0 + min(q0 + 2 * BQ, S) - 1) / BKV + 1 : 0};
   const int ntiles = max(nt[0], nt[1]);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -218,8 +225,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int x = (warp - 2) >> 2;    // query tile of this warpgroup
     const int quarter = warp & 3;     // TMEM lanes 32 quarter .. (fixed by the warp's rank)
     const int r = 32 * quarter + lane;
-    const int qx0 = q0 + BQ * x;
-    const int qpos = qx0 + r;
+    const int qx0 = q0 + BQ * x;  // the tile's first query (its smallest position is p0 + qx0)
+    // this row's query (within the call) and head; rows past the queries are computed but not stored
+    const bool rvalid = packed ? r < grp * S : qx0 + r < S;
+    const int qpos = packed ? (rvalid ? r % S : 0) : qx0 + r;
+    const int hrow = packed ? h + (rvalid ? r / S : 0) : h;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const uint32_t t_o = tmem + T_O + 128 * x + lane_off;
     float m_ref = -INFINITY, l = 0.f;
@@ -287,13 +297,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (ok && nt[x] > 0) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      bf16* orow = out + ((int64_t)b * S + qpos) * ((int64_t)nq * D) + (int64_t)h * D;
+      bf16* orow = out + ((int64_t)b * S + qpos) * ((int64_t)nq * D) + (int64_t)hrow * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float v[32];
         tmem_ld32(t_o + 32 * c, v);
         tc_wait_ld();
-        if (qpos < S) {
+        if (rvalid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
@@ -331,8 +341,9 @@ cudaError_t launch_flash_tc(const void* q, const void* K, const void* V, void* o
   static std::atomic<uint64_t> smem_set{0};
   if (cudaError_t e = set_smem_limit(flash_tc_kernel, SMEM, smem_set); e != cudaSuccess) return e;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-  dim3 grid((unsigned)((S + 2 * BQ - 1) / (2 * BQ)), (unsigned)nq, (unsigned)B);
-  flash_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, (bf16*)o, S, nq, nkv, ctx, start, scale_log2,
+  const int packed = start && (int64_t)S * (nq / nkv) <= BQ;  // a few new tokens: heads of a group share a tile
+  dim3 grid(packed ? 1u : (unsigned)((S + 2 * BQ - 1) / (2 * BQ)), packed ? (unsigned)nkv : (unsigned)nq, (unsigned)B);
+  flash_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, (bf16*)o, S, nq, nkv, ctx, start, packed, scale_log2,
                                                status_ptr());
   return cudaGetLastError();
 }

@@ -35,11 +35,15 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int THREADS = 256;       // skinny kernel: 4 role warps + 4 epilogue warps
 constexpr int GEMM_THREADS = 384;  // main kernel: 4 role warps + 8 epilogue warps (two column halves)
 constexpr int TMEM_COLS = 512;
-constexpr int GROUP_M = 16;  // tile raster: GROUP_M row blocks sweep the N blocks together
+// tile raster: group_m row blocks sweep the N blocks together (the host picks
+// group_m per launch: more row blocks when a row block's A is small, so each
+// W tile is read fewer times while the group's A stays in L2)
+constexpr int GROUP_M_SMALL_K = 32, GROUP_M_LARGE_K = 16;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 
 struct EpiP {
   int M, N;
+  int group_m;  // raster group (row blocks)
   float* c;
   int64_t ldc;
   float* s;
@@ -251,11 +255,11 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, int half, const EpiP
   }
 }
 
-LOOP_DEV void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
-  const int per_group = GROUP_M * num_n;
+LOOP_DEV void tile_coords(int tile, int num_m, int num_n, int group_m, int& mb, int& nb) {
+  const int per_group = group_m * num_n;
   const int g = tile / per_group;
-  const int first = g * GROUP_M;
-  const int gsz = min(num_m - first, GROUP_M);
+  const int first = g * group_m;
+  const int gsz = min(num_m - first, group_m);
   const int r = tile % per_group;
   mb = first + r % gsz;
   nb = r / gsz;
@@ -304,7 +308,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     bool ok = true;
     for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
       int mb, nb;
-      tile_coords(tile, num_m, num_n, mb, nb);
+      tile_coords(tile, num_m, num_n, p.group_m, mb, nb);
       for (int kb = 0; kb < kbs; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, status, STATUS_WAIT_PRODUCER)) { ok = false; break; }
         mbar_expect_tx(&full[stage], STAGE_BYTES);
@@ -346,7 +350,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int acc = local & 1;
       const uint32_t aphase = (local >> 1) & 1;
       int mb, nb;
-      tile_coords(tile, num_m, num_n, mb, nb);
+      tile_coords(tile, num_m, num_n, p.group_m, mb, nb);
       const bool got = mbar_wait(&tfull[acc], aphase, status, STATUS_WAIT_EPILOGUE);
       if (!__all_sync(0xffffffffu, got)) break;  // the whole warp leaves together
       tc_fence_after();
@@ -636,6 +640,7 @@ cudaError_t launch_gemm_tc(const void* A, const void* W, int64_t M, int64_t N, i
   EpiP p{};
   p.M = (int)M;
   p.N = (int)N;
+  p.group_m = K <= 4096 ? GROUP_M_SMALL_K : GROUP_M_LARGE_K;
   p.c = e.c;
   p.ldc = e.ldc;
   p.s = e.s;

@@ -240,13 +240,16 @@ def test_mid_bf16_mixed_length_decode():
         L.loop_model_destroy(g)
 
 
-def test_mid_bf16_extend_after_ragged_prefill():
-    """loop_extend of k = 8 tokens on sequences of different lengths: the
+@pytest.mark.parametrize("k", [8, 32, 33])
+def test_mid_bf16_extend_after_ragged_prefill(k):
+    """loop_extend of k tokens on sequences of different lengths: the
     tensor-core flash kernel with a different start position per sequence
     (keys before the new positions, the causal block among them), each
-    sequence against its own oracle's decode steps."""
-    lens, k = [1100, 77, 530], 8
-    m = dict(W.model_config("tiny_fp32", **MID4), max_batch=3, max_ctx=1120)
+    sequence against its own oracle's decode steps.  With 4 query heads per kv
+    head, k <= 32 runs the packed tile (the group's heads share one 128-row
+    tile; k = 32 fills it) and k = 33 the unpacked one."""
+    lens = [1100, 77, 530]
+    m = dict(W.model_config("tiny_fp32", **MID4), max_batch=3, max_ctx=1100 + k)
     g = L.loop_model_create(L.make_config(**m), seed=12)
     try:
         seqs = [seeded.tokens(70 + i, 1, n, m["vocab"])[0] for i, n in enumerate(lens)]
