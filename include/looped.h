@@ -73,8 +73,22 @@ typedef struct {
   float rope_base, norm_eps;                   /* [1e4, 1e-6] */
   int32_t dtype;                               /* LOOP_F32 or LOOP_BF16 (mHC parameters are always fp32) */
   int32_t io_mode;                             /* LOOP_TOKENS_TO_LOGITS or LOOP_HIDDEN_TO_HIDDEN */
-  int32_t max_batch, max_ctx;                  /* size of the cache arena */
+  int32_t max_batch, max_ctx;                  /* sequences and positions per sequence the caches hold */
+  int32_t kv_pages;                            /* KV pages of 64 positions in each full-attention execution's
+                                                  pool; 0 = max_batch * ceil(max_ctx / 64), enough for every
+                                                  sequence at max_ctx (see "KV cache" below) */
 } loop_config;
+
+/* KV cache.  Each full-attention execution keeps its keys and values in a
+ * pool of pages of 64 positions; one page table per sequence, shared by all
+ * executions (every execution of a sequence holds the same positions), maps
+ * each block of 64 positions to a page.  A prefill (or ragged prefill) of a
+ * sequence returns its pages to the pool and takes what its new length needs;
+ * decode and extend take a page when a sequence crosses a block boundary.  With
+ * kv_pages below max_batch * ceil(max_ctx / 64) the sequences share a smaller
+ * pool (continuous batching of sequences of different lengths); a call whose
+ * sequences would need more pages than are free returns LOOP_ERANGE and
+ * changes nothing. */
 
 typedef struct loop_model loop_model;
 
@@ -131,7 +145,8 @@ LOOP_API int32_t loop_model_create(const loop_config* cfg, const float* const* h
  *   out (the collapsed streams; no embedding, final norm or head).
  * Writes each execution's KV (positions 0..S-1) and final linear-attention
  * state into its own slot; afterwards the sequences have length S.
- * LOOP_ERANGE if B > max_batch or S > max_ctx. */
+ * LOOP_ERANGE if B > max_batch, S > max_ctx or the KV page pool cannot hold
+ * the B sequences. */
 LOOP_API int32_t loop_prefill(loop_model* m, const int32_t* d_tokens, const float* d_hidden, int32_t B, int32_t S,
                      float* d_out, uint32_t flags, void* stream);
 
@@ -145,7 +160,12 @@ LOOP_API int32_t loop_prefill(loop_model* m, const int32_t* d_tokens, const floa
  * of each sequence, processed at its current length; d_logits fp32 [B][vocab].
  * Appends one KV position per full-attention execution, advances every
  * linear-attention state, then adds 1 to each sequence length.
- * LOOP_ERANGE if a sequence would pass max_ctx. */
+ * LOOP_ERANGE if a sequence would pass max_ctx or no KV page is free.
+ * After the first step, a step's kernels are replayed from a CUDA graph
+ * captured on a private stream (one per batch size and 1,024-position context
+ * range; not while per-launch timing or a capture is on): the tokens are copied
+ * into a model buffer first and the logits out of one afterwards, all on
+ * `stream`. */
 LOOP_API int32_t loop_decode_step(loop_model* m, const int32_t* d_tokens, int32_t B, float* d_logits, void* stream);
 
 /* Append k tokens to each of sequences 0..B-1 in one pass: d_tokens int32
@@ -160,7 +180,8 @@ LOOP_API int32_t loop_decode_step(loop_model* m, const int32_t* d_tokens, int32_
  * LOOP_ALL_POSITIONS.  Appends k KV positions per full-attention execution,
  * advances every linear-attention state by k tokens, then adds k to each
  * sequence length.  TOKENS_TO_LOGITS models only (LOOP_EINVAL otherwise);
- * LOOP_ERANGE if a sequence would pass max_ctx, B > max_batch, or B * k
+ * LOOP_ERANGE if a sequence would pass max_ctx, B > max_batch, the KV pages
+ * would run out, or B * k
  * exceeds the model's per-call token budget (max(max_ctx, min(max_batch *
  * max_ctx, 65536)) tokens). */
 LOOP_API int32_t loop_extend(loop_model* m, const int32_t* d_tokens, int32_t B, int32_t k, float* d_out,
@@ -175,7 +196,8 @@ LOOP_API int32_t loop_extend(loop_model* m, const int32_t* d_tokens, int32_t B, 
  * position) or, with LOOP_ALL_POSITIONS, the packed [sum h_lens][vocab].
  * Each sequence runs as its own pass through the same kernels as
  * loop_prefill, so its results equal a loop_prefill of that sequence alone.
- * TOKENS_TO_LOGITS models only; LOOP_ERANGE if b0 + B > max_batch or a length
+ * TOKENS_TO_LOGITS models only; LOOP_ERANGE if the KV pages would run out,
+ * b0 + B > max_batch or a length
  * is outside [1, max_ctx]. */
 LOOP_API int32_t loop_prefill_ragged(loop_model* m, const int32_t* d_tokens, const int32_t* h_lens, int32_t b0,
                                      int32_t B, float* d_out, uint32_t flags, void* stream);

@@ -34,7 +34,7 @@ class loop_config(C.Structure):
         "n_prelude", "n_block", "n_loops", "n_coda", "group", "full_slot", "hidden", "ffn", "vocab",
         "n_q", "n_kv", "head_dim", "n_lin", "lin_dim", "lin_chunk", "n_streams", "sinkhorn_iters")] + [
         ("rope_base", C.c_float), ("norm_eps", C.c_float)] + [
-        (n, C.c_int32) for n in ("dtype", "io_mode", "max_batch", "max_ctx")]
+        (n, C.c_int32) for n in ("dtype", "io_mode", "max_batch", "max_ctx", "kv_pages")]
 
 
 def make_config(**kw) -> loop_config:

@@ -37,7 +37,8 @@ constexpr int DEC_SMEM = DEC_Q_BYTES + DEC_WARPS * DEC_KV_BYTES + DEC_WARPS * DE
 __global__ void __launch_bounds__(DEC_THREADS, 1)
     attn_decode_partial_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                                const bf16* __restrict__ q, const int32_t* __restrict__ start, int nq, int nkv,
-                               int64_t ctx, int nchunks, float scale_log2, float* __restrict__ po,
+                               const int32_t* __restrict__ table, int pps, int nchunks, float scale_log2,
+                               float* __restrict__ po,
                                float* __restrict__ pml, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -51,8 +52,17 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
 
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int L = start[b] + 1;  // keys 0 .. start[b]; the new token's K/V are already in the cache
   const int k0 = chunk * DEC_CHUNK;
+  // The producer looks up the chunk's page rows first, so the loads' latency
+  // passes under the Q staging below (entries past the sequence are read, in
+  // bounds, and not used).
+  int rows[DEC_CHUNK / DEC_TILE];
+  if (warp == DEC_WARPS && lane == 0) {
+#pragma unroll
+    for (int j = 0; j < DEC_CHUNK / DEC_TILE; ++j)
+      rows[j] = (int)kv_row(table, pps, nkv, b, kvh, (int64_t)min(k0 / DEC_TILE + j, pps - 1) * DEC_TILE);
+  }
+  const int L = start[b] + 1;  // keys 0 .. start[b]; the new token's K/V are already in the cache
   const int64_t obase = ((int64_t)b * nq + kvh * DEC_G) * nchunks + chunk;
   if (k0 >= L) {  // past this sequence's end: an empty partial
     if (tid < DEC_G) {
@@ -82,14 +92,15 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     if (lane == 0) {
       prefetch_tmap(&tk);
       prefetch_tmap(&tv);
-      const int64_t row0 = ((int64_t)b * nkv + kvh) * ctx + k0;
-      for (int j = 0; j < ntiles; ++j) {
+#pragma unroll  // unrolled so rows[] stays in registers
+      for (int j = 0; j < DEC_CHUNK / DEC_TILE; ++j) {
+        if (j >= ntiles) break;
         const int s = j % DEC_WARPS;
         const uint32_t ph = (j / DEC_WARPS) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, status, STATUS_WAIT_PRODUCER)) break;
         uint8_t* kt = ring + s * DEC_KV_BYTES;
         uint8_t* vt = kt + DEC_KV_BYTES / 2;
-        const int row = (int)(row0 + (int64_t)j * DEC_TILE);
+        const int row = rows[j];  // a whole page
         mbar_expect_tx(&full[s], DEC_KV_BYTES);
         tma_load_2d(kt, &tk, &full[s], 0, row);
         tma_load_2d(kt + DEC_KV_BYTES / 4, &tk, &full[s], 64, row);
@@ -255,29 +266,33 @@ bool map_rows128(CUtensorMap* m, const void* ptr, int64_t rows, int box_rows) {
 
 bool decode_attention_supported(int hd, int nq, int nkv) { return hd == D && nq == DEC_G * nkv; }
 
+int decode_attention_chunks(int max_len) { return (max_len + DEC_CHUNK - 1) / DEC_CHUNK; }
+
 int64_t decode_attention_scratch_floats(int B, int nq, int64_t ctx) {
   const int64_t nch = (ctx + DEC_CHUNK - 1) / DEC_CHUNK;
   return (int64_t)B * nq * nch * (D + 2);
 }
 
-// q [B][nq][1][128]; K/V cache [B][nkv][ctx][128] with the new position
-// already written; start[b] = position of the new token; o [B][nq*128].
-// scratch: decode_attention_scratch_floats(B, nq, ctx) floats.
+// q [B][nq][1][128]; K/V paged pools of pool_rows rows (see kv_row) with the
+// new position already written; start[b] = position of the new token;
+// o [B][nq*128].  scratch: decode_attention_scratch_floats(B, nq, max_ctx) floats.
 cudaError_t launch_attention_decode(const void* q, const void* K, const void* V, void* o, int B, int nq, int nkv,
-                                    int64_t ctx, int max_len, const int32_t* start, float* scratch, cudaStream_t st) {
+                                    const int32_t* table, int pps, int64_t pool_rows, int max_len,
+                                    const int32_t* start, float* scratch, cudaStream_t st) {
   if (B == 0) return cudaSuccess;
+  static_assert(DEC_TILE == KV_PAGE, "a decode tile is one KV page");
   CUtensorMap mk, mv;
-  if (!map_rows128(&mk, K, (int64_t)B * nkv * ctx, DEC_TILE) || !map_rows128(&mv, V, (int64_t)B * nkv * ctx, DEC_TILE))
+  if (!map_rows128(&mk, K, pool_rows, DEC_TILE) || !map_rows128(&mv, V, pool_rows, DEC_TILE))
     return cudaErrorInvalidValue;
   static std::atomic<uint64_t> smem_set{0};
   if (cudaError_t e = set_smem_limit(attn_decode_partial_kernel, DEC_SMEM, smem_set); e != cudaSuccess) return e;
-  const int nch = (max_len + DEC_CHUNK - 1) / DEC_CHUNK;
+  const int nch = decode_attention_chunks(max_len);
   float* po = scratch;
   float* pml = scratch + (int64_t)B * nq * nch * D;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   dim3 g1((unsigned)nch, (unsigned)nkv, (unsigned)B);
-  attn_decode_partial_kernel<<<g1, DEC_THREADS, DEC_SMEM, st>>>(mk, mv, (const bf16*)q, start, nq, nkv, ctx, nch,
-                                                                scale_log2, po, pml, status_ptr());
+  attn_decode_partial_kernel<<<g1, DEC_THREADS, DEC_SMEM, st>>>(mk, mv, (const bf16*)q, start, nq, nkv, table, pps,
+                                                                nch, scale_log2, po, pml, status_ptr());
   dim3 g2((unsigned)nq, (unsigned)B);
   attn_decode_combine_kernel<<<g2, D, 0, st>>>(po, pml, nq, nch, (bf16*)o);
   return cudaGetLastError();

@@ -100,7 +100,8 @@ LOOP_DEV uint64_t kmajor_desc(uint32_t base, int rows, int kk) {
 __global__ void __launch_bounds__(THREADS, 1)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, bf16* __restrict__ out, int S, int nq, int nkv,
-                    int64_t ctx, const int32_t* __restrict__ start, int packed, float scale_log2, int* status) {
+                    const int32_t* __restrict__ table, int pps, const int32_t* __restrict__ start, int packed,
+                    float scale_log2, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = smem;                 // tile X at sq + X Q_BYTES
@@ -164,13 +165,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_load_2d(sq + x * Q_BYTES, &tq, q_full, 0, qrow + x * BQ);
       tma_load_2d(sq + x * Q_BYTES + Q_BYTES / 2, &tq, q_full, 64, qrow + x * BQ);
     }
-    const int64_t krow0 = ((int64_t)b * nkv + kvh) * ctx;
+    // key tile j is page j; its row is looked up one tile ahead, under the wait
+    int next_row = ntiles > 0 ? (int)kv_row(table, pps, nkv, b, kvh, 0) : 0;
     for (int j = 0; j < ntiles; ++j) {
       const int s = j % NS;
+      const int row = next_row;
+      if (j + 1 < ntiles) next_row = (int)kv_row(table, pps, nkv, b, kvh, (int64_t)(j + 1) * BKV);
       if (!mbar_wait(&kv_empty[s], ((j / NS) & 1) ^ 1, status, STATUS_WAIT_PRODUCER)) break;
       uint8_t* kt = skv + 2 * s * KV_TILE;
       uint8_t* vt = kt + KV_TILE;
-      const int row = (int)(krow0 + (int64_t)j * BKV);
       mbar_expect_tx(&kv_full[s], 2 * KV_TILE);
       tma_load_2d(kt, &tk, &kv_full[s], 0, row);
       tma_load_2d(kt + KV_TILE / 2, &tk, &kv_full[s], 64, row);
@@ -327,24 +330,25 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 bool flash_tc_supported(int hd, int nq, int nkv) { return hd == D && nq % nkv == 0; }
 
-// q [B][nq][S][128], K/V cache [B][nkv][ctx][128], o [B*S][nq*128].  The S
-// queries of sequence b sit at positions start[b] .. start[b] + S - 1 (start
-// NULL: from 0) and their keys, positions 0 .. start[b] + S - 1, are in the
-// cache.
+// q [B][nq][S][128], K/V paged pools of pool_rows rows (see kv_row), o
+// [B*S][nq*128].  The S queries of sequence b sit at positions start[b] ..
+// start[b] + S - 1 (start NULL: from 0) and their keys, positions 0 ..
+// start[b] + S - 1, are in the cache.
 cudaError_t launch_flash_tc(const void* q, const void* K, const void* V, void* o, int B, int S, int nq, int nkv,
-                            int64_t ctx, const int32_t* start, cudaStream_t st) {
+                            const int32_t* table, int pps, int64_t pool_rows, const int32_t* start, cudaStream_t st) {
   if (B == 0 || S == 0) return cudaSuccess;
+  static_assert(BKV == KV_PAGE, "a key tile is one KV page");
   CUtensorMap mq, mk, mv;
-  if (!map_rows128(&mq, q, (int64_t)B * nq * S, BQ) || !map_rows128(&mk, K, (int64_t)B * nkv * ctx, BKV) ||
-      !map_rows128(&mv, V, (int64_t)B * nkv * ctx, BKV))
+  if (!map_rows128(&mq, q, (int64_t)B * nq * S, BQ) || !map_rows128(&mk, K, pool_rows, BKV) ||
+      !map_rows128(&mv, V, pool_rows, BKV))
     return cudaErrorInvalidValue;
   static std::atomic<uint64_t> smem_set{0};
   if (cudaError_t e = set_smem_limit(flash_tc_kernel, SMEM, smem_set); e != cudaSuccess) return e;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   const int packed = start && (int64_t)S * (nq / nkv) <= BQ;  // a few new tokens: heads of a group share a tile
   dim3 grid(packed ? 1u : (unsigned)((S + 2 * BQ - 1) / (2 * BQ)), packed ? (unsigned)nkv : (unsigned)nq, (unsigned)B);
-  flash_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, (bf16*)o, S, nq, nkv, ctx, start, packed, scale_log2,
-                                               status_ptr());
+  flash_tc_kernel<<<grid, THREADS, SMEM, st>>>(mq, mk, mv, (bf16*)o, S, nq, nkv, table, pps, start, packed,
+                                               scale_log2, status_ptr());
   return cudaGetLastError();
 }
 

@@ -77,6 +77,18 @@ LOOP_DEV float log_sigmoidf_(float x) {
 }
 
 // ---------------------------------------------------------------------------
+// Paged KV cache.  The keys (or values) of one full-attention execution live
+// in a pool [pages][n_kv][KV_PAGE][head_dim]; position pos of sequence b is in
+// page table[b * pps + pos / KV_PAGE] (pps = pages per sequence).  kv_row
+// gives the pool row of (b, kv head h, pos).
+// ---------------------------------------------------------------------------
+constexpr int KV_PAGE = 64;
+LOOP_DEV int64_t kv_row(const int32_t* table, int pps, int nkv, int64_t b, int h, int64_t pos) {
+  const int64_t page = table[b * pps + pos / KV_PAGE];
+  return (page * nkv + h) * KV_PAGE + pos % KV_PAGE;
+}
+
+// ---------------------------------------------------------------------------
 // programmatic dependent launch: a kernel launched with the programmatic
 // stream-serialization attribute may start before the previous kernel on its
 // stream ends; it must call griddep_wait() before touching anything that

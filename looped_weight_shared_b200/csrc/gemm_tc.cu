@@ -31,7 +31,9 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int EPI_OFF = STAGES * STAGE_BYTES + 256;  // after the barriers: 8 epilogue warps x 4 KB
+constexpr int SMEM_BYTES = EPI_OFF + 8 * 4096 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 constexpr int THREADS = 256;       // skinny kernel: 4 role warps + 4 epilogue warps
 constexpr int GEMM_THREADS = 384;  // main kernel: 4 role warps + 8 epilogue warps (two column halves)
 constexpr int TMEM_COLS = 512;
@@ -56,7 +58,8 @@ struct EpiP {
   const float2* rope;
   const int32_t* start;
   int S, hq, hkv, n_lin;
-  int64_t ctx;
+  const int32_t* table;  // QKV_FULL: KV page table (the call's first sequence) and its row stride
+  int pps;
   float eps;
 };
 
@@ -124,8 +127,9 @@ LOOP_DEV void head_store_rope(uint32_t t0, bf16* dst, const float2* cs_row, bool
 // them in lockstep, and only the memory accesses of rows >= M are skipped.
 // Two epilogue warpgroups share a tile: `half` 0 takes the first 128
 // columns (or the first head, or gate/up chunks 0-1), `half` 1 the rest.
+// xs: this warp's 4 KB shared-memory tile (used by the residual and mHC-write modes).
 template <Epi MODE>
-LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, int half, const EpiP& p) {
+LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, int half, const EpiP& p, float* xs) {
   const bool valid = row < p.M;
   if constexpr (MODE == Epi::F32) {
 #pragma unroll 1
@@ -144,61 +148,67 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, int half, const EpiP
         for (int j = 0; j < 32 && n + j < p.N; ++j) dst[j] = v[j];
       }
     }
-  } else if constexpr (MODE == Epi::RESID) {
-#pragma unroll 1
-    for (int c = 4 * half; c < 4 * half + 4; ++c) {
-      const int n = n0 + 32 * c;
-      float v[32];
-      ld_chunk(tacc + 32 * c, v);
-      if (!valid) continue;
-      float4* h = reinterpret_cast<float4*>(p.c + (int64_t)row * p.N + n);
-      float4 x[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) x[j] = h[j];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        x[j].x += v[4 * j]; x[j].y += v[4 * j + 1]; x[j].z += v[4 * j + 2]; x[j].w += v[4 * j + 3];
-        h[j] = x[j];
-      }
-    }
-  } else if constexpr (MODE == Epi::MHC_WRITE) {
-    const int crow = valid ? row : 0;
-    const float4 c0 = reinterpret_cast<const float4*>(p.coef + (int64_t)crow * 8)[0];
-    const float4 c1 = reinterpret_cast<const float4*>(p.coef + (int64_t)crow * 8)[1];
-    // c0 = (pre0, pre1, post0, post1), c1 = (res00, res01, res10, res11)
+  } else if constexpr (MODE == Epi::RESID || MODE == Epi::MHC_WRITE) {
+    // Read-modify-write of fp32 rows (the residual, or both mHC streams).  A
+    // thread holds one accumulator row, so the warp first passes each 32 x 32
+    // chunk through its shared-memory tile (16-byte slots XOR-swizzled by row,
+    // conflict-free both ways); then 8 lanes cover one row's 128 contiguous
+    // bytes and every load or store instruction touches 4 rows, not 32.
+    const int lane = threadIdx.x & 31;
+    const int row0 = row - lane;  // the warp's first row
+    float4* xs4 = reinterpret_cast<float4*>(xs);
     const int64_t plane = (int64_t)p.M * p.N;
 #pragma unroll 1
     for (int c = 4 * half; c < 4 * half + 4; ++c) {
       const int n = n0 + 32 * c;
       float v[32];
       ld_chunk(tacc + 32 * c, v);
-      if (!valid) continue;
-      float4* s0 = reinterpret_cast<float4*>(p.s + (int64_t)row * p.N + n);
-      float4* s1 = reinterpret_cast<float4*>(p.s + plane + (int64_t)row * p.N + n);
-      // all loads first: s0 and s1 may alias as far as the compiler knows
-      float4 a[8], b[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) a[j] = __ldcs(s0 + j);
+      for (int j = 0; j < 8; ++j)
+        xs4[lane * 8 + (j ^ (lane & 7))] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      __syncwarp();
+      const int col4 = lane & 7;
+      float4 y[8], a[8], b[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) b[j] = __ldcs(s1 + j);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float4 x, y;
-        x.x = c1.x * a[j].x + c1.y * b[j].x + c0.z * v[4 * j + 0];
-        x.y = c1.x * a[j].y + c1.y * b[j].y + c0.z * v[4 * j + 1];
-        x.z = c1.x * a[j].z + c1.y * b[j].z + c0.z * v[4 * j + 2];
-        x.w = c1.x * a[j].w + c1.y * b[j].w + c0.z * v[4 * j + 3];
-        y.x = c1.z * a[j].x + c1.w * b[j].x + c0.w * v[4 * j + 0];
-        y.y = c1.z * a[j].y + c1.w * b[j].y + c0.w * v[4 * j + 1];
-        y.z = c1.z * a[j].z + c1.w * b[j].z + c0.w * v[4 * j + 2];
-        y.w = c1.z * a[j].w + c1.w * b[j].w + c0.w * v[4 * j + 3];
-        a[j] = x;
-        b[j] = y;
+      for (int k = 0; k < 8; ++k) {
+        const int rr = 4 * k + (lane >> 3);
+        y[k] = xs4[rr * 8 + (col4 ^ (rr & 7))];
+        if (row0 + rr < p.M) {
+          const int64_t off = (int64_t)(row0 + rr) * p.N + n + 4 * col4;
+          if constexpr (MODE == Epi::RESID) {
+            a[k] = *reinterpret_cast<const float4*>(p.c + off);
+          } else {
+            a[k] = __ldcs(reinterpret_cast<const float4*>(p.s + off));
+            b[k] = __ldcs(reinterpret_cast<const float4*>(p.s + plane + off));
+          }
+        }
       }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) s0[j] = a[j];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) s1[j] = b[j];
+      for (int k = 0; k < 8; ++k) {
+        const int rr = 4 * k + (lane >> 3);
+        if (row0 + rr >= p.M) continue;
+        const int64_t off = (int64_t)(row0 + rr) * p.N + n + 4 * col4;
+        if constexpr (MODE == Epi::RESID) {
+          *reinterpret_cast<float4*>(p.c + off) =
+              make_float4(a[k].x + y[k].x, a[k].y + y[k].y, a[k].z + y[k].z, a[k].w + y[k].w);
+        } else {
+          // (pre0, pre1, post0, post1) and (res00, res01, res10, res11) of the row
+          const float4 c0 = __ldg(reinterpret_cast<const float4*>(p.coef + (int64_t)(row0 + rr) * 8));
+          const float4 c1 = __ldg(reinterpret_cast<const float4*>(p.coef + (int64_t)(row0 + rr) * 8) + 1);
+          float4 x, z;
+          x.x = c1.x * a[k].x + c1.y * b[k].x + c0.z * y[k].x;
+          x.y = c1.x * a[k].y + c1.y * b[k].y + c0.z * y[k].y;
+          x.z = c1.x * a[k].z + c1.y * b[k].z + c0.z * y[k].z;
+          x.w = c1.x * a[k].w + c1.y * b[k].w + c0.z * y[k].w;
+          z.x = c1.z * a[k].x + c1.w * b[k].x + c0.w * y[k].x;
+          z.y = c1.z * a[k].y + c1.w * b[k].y + c0.w * y[k].y;
+          z.z = c1.z * a[k].z + c1.w * b[k].z + c0.w * y[k].z;
+          z.w = c1.z * a[k].w + c1.w * b[k].w + c0.w * y[k].w;
+          *reinterpret_cast<float4*>(p.s + off) = x;
+          *reinterpret_cast<float4*>(p.s + plane + off) = z;
+        }
+      }
+      __syncwarp();  // the tile is rewritten by the next chunk
     }
   } else if constexpr (MODE == Epi::SWIGLU) {
     const int F = p.N / 2;
@@ -246,10 +256,11 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, int half, const EpiP
       if (head < p.hq) {
         head_store_rope(t0, p.q + (((int64_t)b * p.hq + head) * p.S + t) * d, cs, valid);
       } else if (head < p.hq + p.hkv) {
-        head_store_rope(t0, p.k + (((int64_t)b * p.hkv + (head - p.hq)) * p.ctx + pos) * d, cs, valid);
+        const int64_t kr = valid ? kv_row(p.table, p.pps, p.hkv, b, head - p.hq, pos) : 0;
+        head_store_rope(t0, p.k + kr * d, cs, valid);
       } else {
-        head_store(t0, p.v + (((int64_t)b * p.hkv + (head - p.hq - p.hkv)) * p.ctx + pos) * d, false, 0.f,
-                   valid);
+        const int64_t vr = valid ? kv_row(p.table, p.pps, p.hkv, b, head - p.hq - p.hkv, pos) : 0;
+        head_store(t0, p.v + vr * d, false, 0.f, valid);
       }
     }
   }
@@ -355,7 +366,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if (!__all_sync(0xffffffffu, got)) break;  // the whole warp leaves together
       tc_fence_after();
       const uint32_t tacc = tmem + acc * BN + ((uint32_t)(32 * q) << 16);
-      epilogue_tile<MODE>(tacc, mb * BM + 32 * q + lane, nb * BN, (warp - 4) >> 2, p);
+      epilogue_tile<MODE>(tacc, mb * BM + 32 * q + lane, nb * BN, (warp - 4) >> 2, p,
+                          reinterpret_cast<float*>(smem + EPI_OFF) + (warp - 4) * 1024);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -656,7 +668,8 @@ cudaError_t launch_gemm_tc(const void* A, const void* W, int64_t M, int64_t N, i
   p.hq = e.heads_q;
   p.hkv = e.heads_kv;
   p.n_lin = e.n_lin;
-  p.ctx = e.cache_ctx;
+  p.table = e.table;
+  p.pps = e.pps;
   p.eps = e.eps;
   switch (e.mode) {
     case Epi::F32: return launch_mode<Epi::F32>(ma, mb, (int)M, (int)N, (int)K, p, st);

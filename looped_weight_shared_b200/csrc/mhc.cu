@@ -611,21 +611,64 @@ cudaError_t launch_rope_table(float2* tab, int64_t ctx, int hd, double base, cud
 // inspection helpers
 // ---------------------------------------------------------------------------
 template <typename T>
-__global__ void cache_to_f32_kernel(const T* src, int B, int nkv, int64_t ctx, int len, int hd, float* dst) {
+__global__ void cache_to_f32_kernel(const T* src, const int32_t* table, int pps, int B, int nkv, int len, int hd,
+                                    float* dst) {
   const int64_t n = (int64_t)B * nkv * len * hd;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t e = i % hd, p = (i / hd) % len, bh = i / ((int64_t)hd * len);
-    dst[i] = to_f(src[(bh * ctx + p) * hd + e]);
+    dst[i] = to_f(src[kv_row(table, pps, nkv, bh / nkv, (int)(bh % nkv), p) * hd + e]);
   }
 }
-cudaError_t launch_cache_to_f32(const void* src, bool bf, int B, int nkv, int64_t ctx, int len, int hd, float* dst,
-                                cudaStream_t st) {
+cudaError_t launch_cache_to_f32(const void* src, bool bf, const int32_t* table, int pps, int B, int nkv, int len,
+                                int hd, float* dst, cudaStream_t st) {
   const int64_t n = (int64_t)B * nkv * len * hd;
   if (n == 0) return cudaSuccess;
   const unsigned g = (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 16);
-  if (bf) cache_to_f32_kernel<bf16><<<g, 256, 0, st>>>((const bf16*)src, B, nkv, ctx, len, hd, dst);
-  else cache_to_f32_kernel<float><<<g, 256, 0, st>>>((const float*)src, B, nkv, ctx, len, hd, dst);
+  if (bf) cache_to_f32_kernel<bf16><<<g, 256, 0, st>>>((const bf16*)src, table, pps, B, nkv, len, hd, dst);
+  else cache_to_f32_kernel<float><<<g, 256, 0, st>>>((const float*)src, table, pps, B, nkv, len, hd, dst);
   return cudaGetLastError();
+}
+
+// rows 0..len-1 of (sequence b, kv head h), 16 bytes per thread
+__global__ void cache_rows_kernel(const uint4* src, const int32_t* table, int pps, int nkv, int b, int h, int len,
+                                  int row16, uint4* dst) {
+  const int64_t n = (int64_t)len * row16;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t p = i / row16, e = i % row16;
+    dst[i] = src[kv_row(table, pps, nkv, b, h, p) * row16 + e];
+  }
+}
+cudaError_t launch_cache_rows(const void* src, size_t esize, const int32_t* table, int pps, int nkv, int b, int h,
+                              int len, int hd, void* dst, cudaStream_t st) {
+  if (len == 0) return cudaSuccess;
+  const int row16 = (int)(hd * esize / 16);
+  const unsigned g = (unsigned)std::min<int64_t>(((int64_t)len * row16 + 255) / 256, 148 * 16);
+  cache_rows_kernel<<<g, 256, 0, st>>>((const uint4*)src, table, pps, nkv, b, h, len, row16, (uint4*)dst);
+  return cudaGetLastError();
+}
+
+// table[idx[i]] = page[i]: the page-table entries a call changes, passed by
+// value so the update is ordered on the stream without a host copy
+constexpr int kTableBatch = 240;
+struct TableSet {
+  int32_t idx[kTableBatch], page[kTableBatch];
+};
+__global__ void table_set_kernel(int32_t* table, TableSet u, int n) {
+  const int i = threadIdx.x;
+  if (i < n) table[u.idx[i]] = u.page[i];
+}
+cudaError_t launch_table_set(int32_t* table, const int32_t* idx, const int32_t* page, int n, cudaStream_t st) {
+  for (int o = 0; o < n; o += kTableBatch) {
+    TableSet u;
+    const int k = std::min(kTableBatch, n - o);
+    for (int i = 0; i < k; ++i) {
+      u.idx[i] = idx[o + i];
+      u.page[i] = page[o + i];
+    }
+    table_set_kernel<<<1, 256, 0, st>>>(table, u, k);
+    if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 template <typename T>

@@ -53,7 +53,7 @@ bool valid(const loop_config* c) {
   if (c->dtype != LOOP_F32 && c->dtype != LOOP_BF16) return false;
   if (c->io_mode != LOOP_TOKENS_TO_LOGITS && c->io_mode != LOOP_HIDDEN_TO_HIDDEN) return false;
   if (c->io_mode == LOOP_TOKENS_TO_LOGITS && c->vocab <= 0) return false;
-  if (c->max_batch <= 0 || c->max_ctx <= 0) return false;
+  if (c->max_batch <= 0 || c->max_ctx <= 0 || c->kv_pages < 0) return false;
   if (!(c->norm_eps >= 0.f) || !(c->rope_base > 0.f)) return false;
   return true;
 }
@@ -156,6 +156,11 @@ int32_t build_table(const loop_config* c, int32_t* table) {
 
 void release(Model& m) {
   if (!m.allocs.empty()) cudaDeviceSynchronize();
+  for (auto& g : m.graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  m.graphs.clear();
+  if (m.cap_stream) cudaStreamDestroy(m.cap_stream);
+  m.cap_stream = nullptr;
   for (void* p : m.allocs) cudaFree(p);
   m.allocs.clear();
   for (auto& t : m.pending) {
@@ -287,16 +292,27 @@ int32_t create_impl(const loop_config* cfg, const float* const* hw, uint64_t see
     LOOP_RC(fill_f32(m, hw, seed, wi, 0, m.sites[s].gamma, 2 * H, true));
     LOOP_RC(fill_f32(m, hw, seed, wi + 1, site_stream(s), m.sites[s].phi, 16 * H, false));
   }
-  // cache arena: one slot per execution
+  // KV cache: one page pool per full-attention execution and one page table
+  // per sequence shared by all of them (every execution of a sequence holds
+  // the same positions)
   const int64_t Bm = c.max_batch, ctx = c.max_ctx;
+  m.pps = (int)((ctx + KV_PAGE - 1) / KV_PAGE);
+  m.n_pages = c.kv_pages > 0 ? c.kv_pages : (int)(Bm * m.pps);
+  const int64_t pool = (int64_t)m.n_pages * nkv * KV_PAGE * hd * es;
   m.kc.assign(m.n_full, nullptr);
   m.vc.assign(m.n_full, nullptr);
   for (int i = 0; i < m.n_full; ++i) {  // zeroed: positions never written hold finite values
-    LOOP_ALLOC(m.kc[i], void*, Bm * nkv * ctx * hd * es);
-    LOOP_ALLOC(m.vc[i], void*, Bm * nkv * ctx * hd * es);
-    LOOP_CU(cudaMemset(m.kc[i], 0, Bm * nkv * ctx * hd * es));
-    LOOP_CU(cudaMemset(m.vc[i], 0, Bm * nkv * ctx * hd * es));
+    LOOP_ALLOC(m.kc[i], void*, pool);
+    LOOP_ALLOC(m.vc[i], void*, pool);
+    LOOP_CU(cudaMemset(m.kc[i], 0, pool));
+    LOOP_CU(cudaMemset(m.vc[i], 0, pool));
   }
+  LOOP_ALLOC(m.d_table, int32_t*, Bm * m.pps * 4);
+  LOOP_CU(cudaMemset(m.d_table, 0, Bm * m.pps * 4));  // unheld blocks point at page 0 (in bounds)
+  m.h_table.assign(Bm * m.pps, 0);
+  m.n_held.assign(Bm, 0);
+  m.free_pages.clear();
+  for (int p = m.n_pages - 1; p >= 0; --p) m.free_pages.push_back(p);
   m.st.assign(m.n_lin, nullptr);
   for (int i = 0; i < m.n_lin; ++i) {
     LOOP_ALLOC(m.st[i], float*, Bm * nl * ld * ld * 4);
@@ -323,6 +339,11 @@ int32_t create_impl(const loop_config* cfg, const float* const* hw, uint64_t see
     for (auto& L : m.L) maxn = std::max(maxn, L.n_in);
     w.cpart_floats = 32 * 64 * maxn;
     LOOP_ALLOC(w.cpart, float*, w.cpart_floats * 4);
+  }
+  if (bf && c.io_mode == LOOP_TOKENS_TO_LOGITS) {  // decode graph input / output
+    LOOP_ALLOC(m.dec_tok, int32_t*, Bm * 4);
+    LOOP_ALLOC(m.dec_logits, float*, Bm * c.vocab * 4);
+    LOOP_CU(cudaStreamCreateWithFlags(&m.cap_stream, cudaStreamNonBlocking));
   }
   if (bf && gla_chunk_supported((int)ld)) {  // one state per SM: the most a segmented prefill uses
     w.gla_seg_floats = 160 * ld * ld;
@@ -411,6 +432,61 @@ void drain_timing(Model& m) {
   m.pending.clear();
 }
 
+// ---- KV pages: a free list on the host; a call's table changes go to the
+// device as kernel arguments, in stream order ----
+int64_t pages_for(int64_t len) { return (len + KV_PAGE - 1) / KV_PAGE; }
+
+// Give sequence b pages for positions [0, len), appending to what it holds
+// (the caller has checked that enough pages are free).
+void pages_grow(Model& m, int b, int64_t len, std::vector<int32_t>& idx, std::vector<int32_t>& pg) {
+  while (m.n_held[b] < pages_for(len)) {
+    const int32_t p = m.free_pages.back();
+    m.free_pages.pop_back();
+    const int32_t i = b * m.pps + m.n_held[b]++;
+    m.h_table[i] = p;
+    idx.push_back(i);
+    pg.push_back(p);
+  }
+}
+
+void pages_release(Model& m, int b) {
+  for (int j = m.n_held[b] - 1; j >= 0; --j) m.free_pages.push_back(m.h_table[b * m.pps + j]);
+  m.n_held[b] = 0;
+}
+
+int32_t pages_upload(Model& m, const std::vector<int32_t>& idx, const std::vector<int32_t>& pg, cudaStream_t st) {
+  if (idx.empty()) return LOOP_OK;
+  LOOP_CU(timed(m, LOOP_K_OTHER, 0.0, (int)((idx.size() + 239) / 240), st,
+                [&] { return launch_table_set(m.d_table, idx.data(), pg.data(), (int)idx.size(), st); }));
+  return LOOP_OK;
+}
+
+// Restart sequences b0 .. b0 + n - 1 at lengths len(i) (their old pages go
+// back first).  LOOP_ERANGE, with nothing changed, if the pool is too small.
+template <typename Len>
+int32_t pages_reset(Model& m, int b0, int n, Len len, cudaStream_t st) {
+  int64_t avail = (int64_t)m.free_pages.size(), need = 0;
+  for (int i = 0; i < n; ++i) {
+    avail += m.n_held[b0 + i];
+    need += pages_for(len(i));
+  }
+  if (need > avail) return fail(LOOP_ERANGE, "KV page pool exhausted");
+  std::vector<int32_t> idx, pg;
+  for (int i = 0; i < n; ++i) pages_release(m, b0 + i);
+  for (int i = 0; i < n; ++i) pages_grow(m, b0 + i, len(i), idx, pg);
+  return pages_upload(m, idx, pg, st);
+}
+
+// Let sequences 0 .. B - 1 grow by k positions.
+int32_t pages_extend(Model& m, int B, int k, cudaStream_t st) {
+  int64_t need = 0;
+  for (int b = 0; b < B; ++b) need += std::max<int64_t>(0, pages_for((int64_t)m.seq_len[b] + k) - m.n_held[b]);
+  if (need > (int64_t)m.free_pages.size()) return fail(LOOP_ERANGE, "KV page pool exhausted");
+  std::vector<int32_t> idx, pg;
+  for (int b = 0; b < B; ++b) pages_grow(m, b, (int64_t)m.seq_len[b] + k, idx, pg);
+  return pages_upload(m, idx, pg, st);
+}
+
 // A projection: C = A W^T followed by its epilogue.
 cudaError_t project(Model& m, const void* A, const void* W, int64_t M, int64_t N, int64_t K, const EpiArgs& e,
                     cudaStream_t st) {
@@ -443,10 +519,13 @@ cudaError_t project(Model& m, const void* A, const void* W, int64_t M, int64_t N
                [&] { return launch_epilogue_unfused(C, ldc, M, N, e, bf16_model(m), st); });
 }
 
-// Causal GQA attention of the current q against this execution's KV slot.
-cudaError_t attention(Model& m, const void* Kc, const void* Vc, int B, int S, const int32_t* d_start, cudaStream_t st) {
+// Causal GQA attention of the current q against this execution's KV page
+// pools; `table` is the page table of the call's first sequence.
+cudaError_t attention(Model& m, const void* Kc, const void* Vc, const int32_t* table, int B, int S,
+                      const int32_t* d_start, cudaStream_t st) {
   const loop_config& c = m.c;
   const bool bf = bf16_model(m);
+  const int64_t pool_rows = (int64_t)m.n_pages * c.n_kv * KV_PAGE;
   // algorithmic FLOPs: QK^T and PV over the causal keys of every query
   double pairs = (double)B * S * (S + 1) / 2.0;
   if (m.extending)
@@ -463,17 +542,18 @@ cudaError_t attention(Model& m, const void* Kc, const void* Vc, int B, int S, co
     }
     const double dflops = 4.0 * keys * c.head_dim * c.n_q;
     return timed(m, LOOP_K_ATTENTION, dflops, 2, st, [&] {
-      return launch_attention_decode(m.w.q, Kc, Vc, m.w.o, B, c.n_q, c.n_kv, c.max_ctx, max_len, d_start,
-                                     m.w.dec_attn, st);
+      return launch_attention_decode(m.w.q, Kc, Vc, m.w.o, B, c.n_q, c.n_kv, table, m.pps, pool_rows, max_len,
+                                     d_start, m.w.dec_attn, st);
     });
   }
   if (bf && S > 1 && flash_tc_supported(c.head_dim, c.n_q, c.n_kv))  // prefill from 0, or extend from seq_len
     return timed(m, LOOP_K_ATTENTION, flops, 1, st, [&] {
-      return launch_flash_tc(m.w.q, Kc, Vc, m.w.o, B, S, c.n_q, c.n_kv, c.max_ctx, m.extending ? d_start : nullptr,
-                             st);
+      return launch_flash_tc(m.w.q, Kc, Vc, m.w.o, B, S, c.n_q, c.n_kv, table, m.pps, pool_rows,
+                             m.extending ? d_start : nullptr, st);
     });
   return timed(m, LOOP_K_ATTENTION, flops, 1, st, [&] {
-    return launch_attention_simple(m.w.q, Kc, Vc, m.w.o, bf, B, S, c.n_q, c.n_kv, c.head_dim, c.max_ctx, d_start, st);
+    return launch_attention_simple(m.w.q, Kc, Vc, m.w.o, bf, B, S, c.n_q, c.n_kv, c.head_dim, table, m.pps, d_start,
+                                   st);
   });
 }
 
@@ -517,14 +597,13 @@ cudaError_t capture(Model& m, const Capture& cp, bool full, const void* Kc, cons
     // K, V of the kv heads of those query heads, positions 0 .. start + S - 1 of the call
     const int64_t grp = c.n_q / c.n_kv, kh0 = h0 / grp, nk = (h0 + n - 1) / grp - kh0 + 1;
     const int64_t len = (m.extending || m.decoding) ? (int64_t)m.seq_len[0] + S : S;
-    for (int64_t j = 0; j < nk; ++j) {
-      const int64_t off = ((kh0 + j) * c.max_ctx) * d * es;
+    for (int64_t j = 0; j < nk; ++j) {  // gathered from sequence 0's pages
       if (cp.k)
-        if (cudaError_t e = cudaMemcpyAsync((char*)cp.k + j * len * d * es, (const char*)Kc + off, len * d * es,
-                                            cudaMemcpyDeviceToDevice, st); e != cudaSuccess) return e;
+        if (cudaError_t e = launch_cache_rows(Kc, es, m.d_table, m.pps, c.n_kv, 0, (int)(kh0 + j), (int)len, (int)d,
+                                              (char*)cp.k + j * len * d * es, st); e != cudaSuccess) return e;
       if (cp.v)
-        if (cudaError_t e = cudaMemcpyAsync((char*)cp.v + j * len * d * es, (const char*)Vc + off, len * d * es,
-                                            cudaMemcpyDeviceToDevice, st); e != cudaSuccess) return e;
+        if (cudaError_t e = launch_cache_rows(Vc, es, m.d_table, m.pps, c.n_kv, 0, (int)(kh0 + j), (int)len, (int)d,
+                                              (char*)cp.v + j * len * d * es, st); e != cudaSuccess) return e;
     }
   } else {
     if (cp.k)
@@ -603,15 +682,16 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
       }
       if (sub == 0) {
         if (kind == LOOP_KIND_FULL) {
-          void* Kc = (char*)m.kc[slot] + (int64_t)b0 * nkv * c.max_ctx * hd * es;
-          void* Vc = (char*)m.vc[slot] + (int64_t)b0 * nkv * c.max_ctx * hd * es;
+          void* Kc = m.kc[slot];
+          void* Vc = m.vc[slot];
+          const int32_t* table = m.d_table + (int64_t)b0 * m.pps;
           EpiArgs qe;
           qe.mode = Epi::QKV_FULL;
           qe.q = w.q; qe.k = Kc; qe.v = Vc;
           qe.rope = m.rope; qe.start = d_start; qe.S = S;
-          qe.heads_q = (int)nq; qe.heads_kv = (int)nkv; qe.hd = (int)hd; qe.cache_ctx = c.max_ctx;
+          qe.heads_q = (int)nq; qe.heads_kv = (int)nkv; qe.hd = (int)hd; qe.table = table; qe.pps = m.pps;
           LOOP_CU(project(m, w.xh, L.w_in, T, L.n_in, H, qe, st));
-          LOOP_CU(attention(m, Kc, Vc, B, S, d_start, st));
+          LOOP_CU(attention(m, Kc, Vc, table, B, S, d_start, st));
           for (const Capture& cp : m.captures)
             if (cp.exec == e && b0 == 0) LOOP_CU(capture(m, cp, true, Kc, Vc, S, st));
         } else {
@@ -652,6 +732,57 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
   le.ldc = c.vocab;
   LOOP_CU(project(m, w.xh, m.embed, rows, c.vocab, H, le, st));
   return LOOP_OK;
+}
+
+// A decode step from a CUDA graph: the step's launches, captured once per
+// (batch, decode-attention chunk count) on a private stream, replayed on the
+// caller's stream between a copy of the tokens in and of the logits out.
+// Returns false (nothing launched) when the step must run eagerly: per-launch
+// timing is on, a loop_capture is armed, no eager step has set up the kernels
+// yet, or capture failed.
+bool decode_graph(Model& m, const int32_t* d_tokens, int B, float* d_logits, cudaStream_t st, int32_t* rc) {
+  if (m.timing || !m.decoded_eagerly || !m.cap_stream || !m.dec_tok || !m.dec_logits || !m.captures.empty())
+    return false;
+  int max_len = 0;
+  for (int b = 0; b < B; ++b) max_len = std::max(max_len, m.seq_len[b] + 1);
+  const int nch = decode_attention_chunks(max_len);
+  Model::DecodeGraph* g = nullptr;
+  for (auto& x : m.graphs)
+    if (x.B == B && x.nch == nch) g = &x;
+  if (!g) {
+    Model::DecodeGraph ng;
+    ng.B = B;
+    ng.nch = nch;
+    const int64_t l0 = m.launches;
+    cudaGraph_t graph = nullptr;
+    if (cudaStreamBeginCapture(m.cap_stream, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    m.decoding = true;
+    const int32_t frc = forward(m, m.dec_tok, nullptr, 0, B, 1, m.d_seq_len, m.dec_logits, 0, true, m.cap_stream);
+    m.decoding = false;
+    const cudaError_t ec = cudaStreamEndCapture(m.cap_stream, &graph);
+    ng.kernels = m.launches - l0;  // what the graph launches; capturing launched nothing
+    m.launches = l0;
+    bool ok = frc == LOOP_OK && ec == cudaSuccess && graph;
+    if (ok) ok = cudaGraphInstantiate(&ng.exec, graph, 0) == cudaSuccess;
+    if (graph) cudaGraphDestroy(graph);
+    if (!ok) {
+      cudaGetLastError();
+      if (ng.exec) cudaGraphExecDestroy(ng.exec);
+      return false;
+    }
+    m.graphs.push_back(ng);
+    g = &m.graphs.back();
+  }
+  cudaError_t e = cudaMemcpyAsync(m.dec_tok, d_tokens, (size_t)B * 4, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = cudaGraphLaunch(g->exec, st);
+  m.launches += g->kernels;
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(d_logits, m.dec_logits, (size_t)B * m.c.vocab * 4, cudaMemcpyDeviceToDevice, st);
+  *rc = e == cudaSuccess ? LOOP_OK : fail(LOOP_ECUDA, std::string("decode graph: ") + cudaGetErrorString(e));
+  return true;
 }
 
 }  // namespace
@@ -701,6 +832,7 @@ int32_t loop_prefill(loop_model* mp, const int32_t* d_tokens, const float* d_hid
   if (c.io_mode == LOOP_TOKENS_TO_LOGITS && !d_tokens) return fail(LOOP_EINVAL, "d_tokens is NULL");
   if (c.io_mode == LOOP_HIDDEN_TO_HIDDEN && !d_hidden) return fail(LOOP_EINVAL, "d_hidden is NULL");
   cudaStream_t st = (cudaStream_t)stream;
+  if (int32_t rc = pages_reset(m, 0, B, [&](int) { return (int64_t)S; }, st); rc != LOOP_OK) return rc;
   const int64_t nl = c.n_lin, ld = c.lin_dim, H = c.hidden;
   const int group = (int)std::max<int64_t>(1, std::min<int64_t>(B, m.w.t_max / S));
   const bool all = flags & LOOP_ALL_POSITIONS;
@@ -730,9 +862,14 @@ int32_t loop_decode_step(loop_model* mp, const int32_t* d_tokens, int32_t B, flo
   for (int b = 0; b < B; ++b)
     if (m.seq_len[b] + 1 > m.c.max_ctx) return fail(LOOP_ERANGE, "sequence would pass max_ctx");
   cudaStream_t st = (cudaStream_t)stream;
-  m.decoding = true;
-  const int32_t rc = forward(m, d_tokens, nullptr, 0, B, 1, m.d_seq_len, d_logits, 0, true, st);
-  m.decoding = false;
+  if (int32_t rc = pages_extend(m, B, 1, st); rc != LOOP_OK) return rc;
+  int32_t rc = LOOP_EINVAL;
+  if (!decode_graph(m, d_tokens, B, d_logits, st, &rc)) {  // eager: per-launch timing, first step, no graph
+    m.decoding = true;
+    rc = forward(m, d_tokens, nullptr, 0, B, 1, m.d_seq_len, d_logits, 0, true, st);
+    m.decoding = false;
+    if (rc == LOOP_OK) m.decoded_eagerly = true;
+  }
   if (rc != LOOP_OK) return rc;
   LOOP_CU(timed(m, LOOP_K_OTHER, 0.0, 1, st, [&] { return launch_advance(m.d_seq_len, B, st); }));
   for (int b = 0; b < B; ++b) m.seq_len[b] += 1;
@@ -750,6 +887,7 @@ int32_t loop_extend(loop_model* mp, const int32_t* d_tokens, int32_t B, int32_t 
   for (int b = 0; b < B; ++b)
     if ((int64_t)m.seq_len[b] + k > m.c.max_ctx) return fail(LOOP_ERANGE, "sequence would pass max_ctx");
   cudaStream_t st = (cudaStream_t)stream;
+  if (int32_t rc = pages_extend(m, B, k, st); rc != LOOP_OK) return rc;
   // the positions of sequence b are seq_len[b] .. seq_len[b] + k - 1: every kernel takes
   // its start from d_seq_len, and attention uses the kernel that honours per-sequence starts
   m.extending = true;
@@ -772,6 +910,7 @@ int32_t loop_prefill_ragged(loop_model* mp, const int32_t* d_tokens, const int32
   for (int i = 0; i < B; ++i)
     if (h_lens[i] < 1 || h_lens[i] > c.max_ctx) return fail(LOOP_ERANGE, "a length is outside [1, max_ctx]");
   cudaStream_t st = (cudaStream_t)stream;
+  if (int32_t rc = pages_reset(m, b0, B, [&](int i) { return (int64_t)h_lens[i]; }, st); rc != LOOP_OK) return rc;
   const int64_t nl = c.n_lin, ld = c.lin_dim;
   const bool all = flags & LOOP_ALL_POSITIONS;
   int64_t off = 0;
@@ -830,8 +969,9 @@ int32_t loop_cache_read(loop_model* mp, int32_t kind, int32_t slot, int32_t B, i
   if (kind == LOOP_KIND_FULL) {
     if (slot < 0 || slot >= m.n_full || len < 0 || len > c.max_ctx) return fail(LOOP_EINVAL, "bad slot or len");
     const int64_t n = (int64_t)B * c.n_kv * len * c.head_dim;
-    LOOP_CU(launch_cache_to_f32(m.kc[slot], bf16_model(m), B, c.n_kv, c.max_ctx, len, c.head_dim, d_out, st));
-    LOOP_CU(launch_cache_to_f32(m.vc[slot], bf16_model(m), B, c.n_kv, c.max_ctx, len, c.head_dim, d_out + n, st));
+    LOOP_CU(launch_cache_to_f32(m.kc[slot], bf16_model(m), m.d_table, m.pps, B, c.n_kv, len, c.head_dim, d_out, st));
+    LOOP_CU(launch_cache_to_f32(m.vc[slot], bf16_model(m), m.d_table, m.pps, B, c.n_kv, len, c.head_dim, d_out + n,
+                                st));
     return LOOP_OK;
   }
   if (kind != LOOP_KIND_LINEAR || slot < 0 || slot >= m.n_lin) return fail(LOOP_EINVAL, "bad kind or slot");

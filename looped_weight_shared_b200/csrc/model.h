@@ -46,14 +46,15 @@ struct EpiArgs {
   const float* coef = nullptr;  // MHC_WRITE: [M][8]
   void* a = nullptr;            // SWIGLU output [M][F]
   void* q = nullptr;            // QKV: q [B][heads][S][d]
-  void* k = nullptr;            // QKV_LINEAR: k; QKV_FULL: K cache base (sequence b0)
-  void* v = nullptr;            // QKV_LINEAR: v; QKV_FULL: V cache base
+  void* k = nullptr;            // QKV_LINEAR: k; QKV_FULL: this execution's K page pool
+  void* v = nullptr;            // QKV_LINEAR: v; QKV_FULL: V page pool
   float* gl = nullptr;          // QKV_LINEAR: log-gates [B][n_lin][S]
   const float2* rope = nullptr; // QKV_FULL: (cos, sin) [max_ctx][hd/2]
   const int32_t* start = nullptr;  // QKV_FULL: start position of each sequence
   int S = 1;                    // tokens per sequence in this call
   int heads_q = 0, heads_kv = 0, hd = 0;
-  int64_t cache_ctx = 0;        // QKV_FULL: max_ctx (position stride of the cache)
+  const int32_t* table = nullptr;  // QKV_FULL: KV page table of the call's first sequence
+  int pps = 0;                     // QKV_FULL: pages per sequence (table row stride)
   int n_lin = 0;
   float eps = 1e-6f;
 };
@@ -132,7 +133,13 @@ struct Model {
   float* final_gain = nullptr;
   std::vector<LayerW> L;
   std::vector<SiteW> sites;
-  std::vector<void*> kc, vc;    // per full-attention slot [max_batch][n_kv][max_ctx][hd]
+  std::vector<void*> kc, vc;    // per full-attention slot: page pool [n_pages][n_kv][KV_PAGE][hd]
+  int pps = 0;                  // KV pages per sequence: ceil(max_ctx / KV_PAGE)
+  int n_pages = 0;              // pages in each execution's pool
+  int32_t* d_table = nullptr;   // [max_batch][pps] page of each block of KV_PAGE positions (all slots)
+  std::vector<int32_t> h_table; // host copy
+  std::vector<int32_t> n_held;  // pages each sequence holds
+  std::vector<int32_t> free_pages;
   std::vector<float*> st;       // per linear slot [max_batch][n_lin][d][d] fp32
   int32_t* d_seq_len = nullptr;
   std::vector<int32_t> seq_len;
@@ -143,6 +150,18 @@ struct Model {
   bool decoding = false;        // inside loop_decode_step: projections use the decode GEMM
   bool extending = false;       // inside loop_extend: sequences start past 0 (attention starts at seq_len)
   std::vector<Capture> captures;
+  // decode steps replayed from CUDA graphs: one graph per (batch, decode-
+  // attention chunk count), captured on a private stream after one eager step
+  struct DecodeGraph {
+    int B = 0, nch = 0;
+    int64_t kernels = 0;
+    cudaGraphExec_t exec = nullptr;
+  };
+  std::vector<DecodeGraph> graphs;
+  cudaStream_t cap_stream = nullptr;
+  bool decoded_eagerly = false;
+  int32_t* dec_tok = nullptr;   // [max_batch] the step's tokens (graph input)
+  float* dec_logits = nullptr;  // [max_batch][vocab] the step's logits (graph output)
 };
 
 bool bf16_model(const Model& m);
@@ -186,13 +205,19 @@ cudaError_t launch_gemm_simt(const void* A, const void* W, bool bf16, int64_t M,
 cudaError_t launch_epilogue_unfused(const float* C, int64_t ldc, int64_t M, int64_t N, const EpiArgs& e, bool bf16,
                                     cudaStream_t st, int splits = 1);
 cudaError_t launch_attention_simple(const void* q, const void* K, const void* V, void* o, bool bf16, int B, int S,
-                                    int nq, int nkv, int hd, int64_t cache_ctx, const int32_t* start,
+                                    int nq, int nkv, int hd, const int32_t* table, int pps, const int32_t* start,
                                     cudaStream_t st);
 cudaError_t launch_gla_recurrent(const void* q, const void* k, const void* v, const float* gl, float* state, void* o,
                                  bool bf16, int B, int S, int nh, int d, cudaStream_t st);
 cudaError_t launch_rope_table(float2* tab, int64_t ctx, int hd, double base, cudaStream_t st);
-cudaError_t launch_cache_to_f32(const void* src, bool bf16, int B, int nkv, int64_t ctx, int len, int hd,
-                                float* dst, cudaStream_t st);
+// K or V of sequences 0..B-1, positions 0..len-1 -> dst fp32 [B][nkv][len][hd]
+cudaError_t launch_cache_to_f32(const void* src, bool bf16, const int32_t* table, int pps, int B, int nkv, int len,
+                                int hd, float* dst, cudaStream_t st);
+// K or V rows 0..len-1 of sequence b, kv head h -> dst [len][hd] in the model dtype
+cudaError_t launch_cache_rows(const void* src, size_t esize, const int32_t* table, int pps, int nkv, int b, int h,
+                              int len, int hd, void* dst, cudaStream_t st);
+// set table[idx[i]] = page[i] for n entries (passed by value)
+cudaError_t launch_table_set(int32_t* table, const int32_t* idx, const int32_t* page, int n, cudaStream_t st);
 cudaError_t launch_advance(int32_t* seq_len, int B, cudaStream_t st, int by = 1);
 cudaError_t launch_selftest_timeout(uint64_t limit_ns, int* result, cudaStream_t st);
 cudaError_t launch_set_len(int32_t* seq_len, int B, int S, cudaStream_t st);
@@ -203,13 +228,15 @@ cudaError_t launch_weight_to_f32(const void* src, bool bf16, int64_t rows, int64
 // at positions start[b] .. (start NULL: from 0)
 bool flash_tc_supported(int hd, int nq, int nkv);
 cudaError_t launch_flash_tc(const void* q, const void* K, const void* V, void* o, int B, int S, int nq, int nkv,
-                            int64_t ctx, const int32_t* start, cudaStream_t st);
+                            const int32_t* table, int pps, int64_t pool_rows, const int32_t* start, cudaStream_t st);
 
-// decode attention (flash-decoding over 128-key chunks; bf16, head_dim 128, group 4)
+// decode attention (flash-decoding over 1024-key chunks; bf16, head_dim 128, group 4)
 bool decode_attention_supported(int hd, int nq, int nkv);
+int decode_attention_chunks(int max_len);  // grid width for the longest sequence
 int64_t decode_attention_scratch_floats(int B, int nq, int64_t ctx);
 cudaError_t launch_attention_decode(const void* q, const void* K, const void* V, void* o, int B, int nq, int nkv,
-                                    int64_t ctx, int max_len, const int32_t* start, float* scratch, cudaStream_t st);
+                                    const int32_t* table, int pps, int64_t pool_rows, int max_len,
+                                    const int32_t* start, float* scratch, cudaStream_t st);
 
 // chunked gated linear attention for prefill (bf16, d = 128)
 bool gla_chunk_supported(int d);

@@ -148,7 +148,7 @@ __global__ void epi_qkv_linear_kernel(CView C, int64_t M, int S, int nh, int d, 
 // one warp per (token, head) over q heads, then k heads, then v heads
 template <typename T>
 __global__ void epi_qkv_full_kernel(CView C, int64_t M, int S, int nq, int nkv, int hd, const float2* rope,
-                                    const int32_t* start, int64_t ctx, T* q, T* K, T* V) {
+                                    const int32_t* start, const int32_t* table, int pps, T* q, T* K, T* V) {
   const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int nheads = nq + 2 * nkv;
@@ -164,9 +164,9 @@ __global__ void epi_qkv_full_kernel(CView C, int64_t M, int S, int nq, int nkv, 
   if (h < nq) {
     dst = q + ((b * nq + h) * S + t) * hd;
   } else if (h < nq + nkv) {
-    dst = K + ((b * nkv + (h - nq)) * ctx + pos) * hd;
+    dst = K + kv_row(table, pps, nkv, b, h - nq, pos) * hd;
   } else {
-    dst = V + ((b * nkv + (h - nq - nkv)) * ctx + pos) * hd;
+    dst = V + kv_row(table, pps, nkv, b, h - nq - nkv, pos) * hd;
     rot = false;
   }
   for (int i = lane; i < half; i += 32) {
@@ -217,10 +217,10 @@ cudaError_t launch_epilogue_unfused(const float* C, int64_t ldc, int64_t M, int6
       const unsigned g = (unsigned)((warps * 32 + 255) / 256);
       if (bf)
         epi_qkv_full_kernel<bf16><<<g, 256, 0, st>>>(cv, M, e.S, e.heads_q, e.heads_kv, e.hd, e.rope, e.start,
-                                                     e.cache_ctx, (bf16*)e.q, (bf16*)e.k, (bf16*)e.v);
+                                                     e.table, e.pps, (bf16*)e.q, (bf16*)e.k, (bf16*)e.v);
       else
         epi_qkv_full_kernel<float><<<g, 256, 0, st>>>(cv, M, e.S, e.heads_q, e.heads_kv, e.hd, e.rope, e.start,
-                                                      e.cache_ctx, (float*)e.q, (float*)e.k, (float*)e.v);
+                                                      e.table, e.pps, (float*)e.q, (float*)e.k, (float*)e.v);
       break;
     }
   }
@@ -229,11 +229,11 @@ cudaError_t launch_epilogue_unfused(const float* C, int64_t ldc, int64_t M, int6
 
 // ---------------------------------------------------------------------------
 // causal GQA attention, one warp per (sequence, q head, query); online softmax
-// q [B][nq][S][hd]; K, V cache [B][nkv][ctx][hd]; o [B*S][nq*hd]
+// q [B][nq][S][hd]; K, V paged caches (see kv_row); o [B*S][nq*hd]
 // ---------------------------------------------------------------------------
 template <typename T, int EPL>
 __global__ void attention_simple_kernel(const T* q, const T* K, const T* V, T* o, int B, int S, int nq, int nkv,
-                                        int64_t ctx, const int32_t* start) {
+                                        const int32_t* table, int pps, const int32_t* start) {
   const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int hd = EPL * 32;
@@ -251,19 +251,18 @@ __global__ void attention_simple_kernel(const T* q, const T* K, const T* V, T* o
     qv[i] = to_f(qr[lane + 32 * i]) * scale;
     acc[i] = 0.f;
   }
-  const T* Kb = K + ((int64_t)b * nkv + kh) * ctx * hd;
-  const T* Vb = V + ((int64_t)b * nkv + kh) * ctx * hd;
   float m = -INFINITY, l = 0.f;
   for (int64_t j = 0; j <= pos; ++j) {
+    const int64_t kr = kv_row(table, pps, nkv, b, kh, j) * hd;
     float sc = 0.f;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) sc += qv[i] * to_f(Kb[j * hd + lane + 32 * i]);
+    for (int i = 0; i < EPL; ++i) sc += qv[i] * to_f(K[kr + lane + 32 * i]);
     sc = warp_sum(sc);
     const float mn = fmaxf(m, sc);
     const float corr = __expf(m - mn), p = __expf(sc - mn);
     l = l * corr + p;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) acc[i] = acc[i] * corr + p * to_f(Vb[j * hd + lane + 32 * i]);
+    for (int i = 0; i < EPL; ++i) acc[i] = acc[i] * corr + p * to_f(V[kr + lane + 32 * i]);
     m = mn;
   }
   T* orow = o + ((int64_t)b * S + t) * nq * hd + (int64_t)h * hd;
@@ -272,17 +271,18 @@ __global__ void attention_simple_kernel(const T* q, const T* K, const T* V, T* o
 }
 
 cudaError_t launch_attention_simple(const void* q, const void* K, const void* V, void* o, bool bf, int B, int S,
-                                    int nq, int nkv, int hd, int64_t ctx, const int32_t* start, cudaStream_t st) {
+                                    int nq, int nkv, int hd, const int32_t* table, int pps, const int32_t* start,
+                                    cudaStream_t st) {
   const int64_t warps = (int64_t)B * nq * S;
   if (warps == 0) return cudaSuccess;
   const unsigned g = (unsigned)((warps * 32 + 255) / 256);
 #define LOOP_ATT(EPL)                                                                                            \
   if (bf)                                                                                                        \
     attention_simple_kernel<bf16, EPL><<<g, 256, 0, st>>>((const bf16*)q, (const bf16*)K, (const bf16*)V,       \
-                                                          (bf16*)o, B, S, nq, nkv, ctx, start);                  \
+                                                          (bf16*)o, B, S, nq, nkv, table, pps, start);           \
   else                                                                                                           \
     attention_simple_kernel<float, EPL><<<g, 256, 0, st>>>((const float*)q, (const float*)K, (const float*)V,    \
-                                                           (float*)o, B, S, nq, nkv, ctx, start);
+                                                           (float*)o, B, S, nq, nkv, table, pps, start);
   switch (hd) {
     case 32: LOOP_ATT(1); break;
     case 64: LOOP_ATT(2); break;

@@ -42,6 +42,7 @@ typedef struct {
   int32_t dtype;   /* 0 = fp32 everywhere, 1 = bf16 weights and GEMM operands */
   int32_t io_mode; /* 0 = tokens -> logits, 1 = hidden -> hidden             */
   int32_t max_batch, max_ctx;
+  int32_t kv_pages; /* the library's KV page-pool size; the oracle keeps a dense cache and ignores it */
 } oracle_config;
 
 enum { ORACLE_FULL = 1, ORACLE_LINEAR = 0 };

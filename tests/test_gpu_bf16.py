@@ -268,3 +268,61 @@ def test_mid_bf16_extend_after_ragged_prefill(k):
         assert L.loop_device_status() == 0
     finally:
         L.loop_model_destroy(g)
+
+
+def test_mid_bf16_paged_kv_pool_shared_by_sequences():
+    """A KV page pool smaller than max_batch x max_ctx, shared by sequences of
+    different lengths: ragged prefills that release and take pages (so a
+    sequence's pages end up scattered over the pool), decode steps that cross
+    64-position page boundaries, a re-prefill of one sequence, and a prefill
+    that would need more pages than are free (LOOP_ERANGE, nothing changed).
+    Every sequence against its own oracle (a dense cache)."""
+    m = dict(W.model_config("tiny_fp32", **MID4), max_batch=4, max_ctx=600, kv_pages=20)
+    V = m["vocab"]
+    g = L.loop_model_create(L.make_config(**m), seed=13)
+    try:
+        om = dict(m, max_batch=1)
+        os_ = [oracle.Model(oracle.make_config(**om), seed=13) for _ in range(3)]
+        lens = [126, 200, 63]  # 2 + 4 + 1 pages
+        seqs = [seeded.tokens(80 + b, 1, n, V)[0] for b, n in enumerate(lens)]
+        ref = np.concatenate([o.prefill(s[None, :]) for o, s in zip(os_, seqs)])
+        out = torch.empty((3, V), device="cuda")
+        L.loop_prefill_ragged(g, torch.from_numpy(np.concatenate(seqs)).cuda(), lens, out)
+        torch.cuda.synchronize()
+        check(out.cpu().numpy(), ref)
+
+        def decode(step):
+            tok = seeded.tokens(90 + step, 1, 3, V, stream=seeded.S_DECODE_TOKENS)[0]
+            d = torch.empty((3, V), device="cuda")
+            L.loop_decode_step(g, torch.from_numpy(tok).cuda(), d)
+            torch.cuda.synchronize()
+            r = np.concatenate([o.decode_step(np.array([t], dtype=np.int32)) for o, t in zip(os_, tok)])
+            check(d.cpu().numpy(), r)
+
+        for step in range(3):  # sequence 0 crosses 128, sequence 2 crosses 64
+            decode(step)
+        # sequence 1 again, longer: its 4 pages go back, 8 are taken (some of them freed ones)
+        s1 = seeded.tokens(85, 1, 450, V)[0]
+        r1 = os_[1].prefill(s1[None, :])
+        o1 = torch.empty((1, V), device="cuda")
+        L.loop_prefill_ragged(g, torch.from_numpy(s1).cuda(), [450], o1, b0=1)
+        torch.cuda.synchronize()
+        check(o1.cpu().numpy(), r1)
+        for step in range(3, 5):
+            decode(step)
+        # 3 + 8 + 2 pages held, 7 free: a 500-token sequence (8 pages) does not fit
+        with pytest.raises(L.LoopError) as err:
+            L.loop_prefill_ragged(g, torch.from_numpy(seeded.tokens(86, 1, 500, V)[0]).cuda(), [500],
+                                  torch.empty((1, V), device="cuda"), b0=3)
+        assert err.value.code == L.LOOP_ERANGE
+        decode(5)
+        # the paged cache read back in position order
+        kv = torch.empty((2, 1, 2, lens[0] + 6, 128), device="cuda")
+        L.loop_cache_read(g, L.LOOP_KIND_FULL, 1, 1, lens[0] + 6, kv)
+        torch.cuda.synchronize()
+        k_ref, v_ref = os_[0].kv(1, 1, lens[0] + 6)
+        check(kv[0].cpu().numpy(), k_ref)
+        check(kv[1].cpu().numpy(), v_ref)
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
