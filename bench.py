@@ -31,11 +31,13 @@ from seeded import workloads as W  # noqa: E402
 DEFAULT_WORKLOAD = "loop9b_prefill_b4_s8192"
 
 # DRAM read + write per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
-# taken under the small-capture rule; None until taken for the current kernel:
-# - tcgen05 GEMM: per launch of the 9B prefill (see profiles/)
+# taken under the capture rules; set to None when the kernel changes:
+# - tcgen05 GEMM: mean over five consecutive full-size launches of the 9B
+#   prefill (SwiGLU, mHC write at K 12,288 and 4,096, q/k/v/gate; one-pass
+#   metrics, see profiles/launches_loop9b_prefill_b4_s8192.md)
 # - decode attention: 1.085 GB per launch on the probe_decode_b64_ctx4096
 #   workload (64 x 4096 keys), scaled by keys to 32,787
-GEMM_TRAFFIC_PER_LAUNCH = None
+GEMM_TRAFFIC_PER_LAUNCH = 3.32e9
 DECODE_ATTN_TRAFFIC_PER_LAUNCH = 1.085e9 * 32787 / 4097
 LONG_WORKLOAD = "loop9b_prefill_b1_s262144"
 EXTEND_K = 8  # tokens per sequence of the timed loop_extend steps
