@@ -481,7 +481,9 @@ def oracle_sample(a, steps=1):
             o.prefill(tok)
             times.append(time.time() - t)
         units = s_tok
-        sample = f"prefill of 1 x {s_tok} tokens of the workload's model (the workload is {w['batch']} x {w['seq']})"
+        sample = (f"prefill of 1 x {s_tok} tokens of the workload's model (the workload is {w['batch']} x {w['seq']}); "
+                  f"a sample, not an extrapolation: at {s_tok} tokens attention is a negligible share of the oracle's "
+                  f"work, at {w['seq']} it is not")
     o.close()
     return dict(value=units / statistics.mean(times), times=times, sample=sample, setup_s=setup,
                 cores=int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)))

@@ -222,18 +222,19 @@ cudaError_t launch_sinkhorn(const float* l, float* out, int64_t count, int n, in
 //
 // (A) mhc_partial: the flattened stream vector u = (s_0, s_1) of a token has
 //     2H entries, cut into `parts` equal parts (2 for long inputs; more when
-//     few tokens must still spread over many SMs); CTA (blk, part) keeps its
-//     part of Phi and gamma in shared memory and every warp streams 8 tokens
-//     of that part with float4 loads, so each Phi value read is used 8 times.
-//     It writes, per token and part, the 8 partial projections
-//     sum_i s_i gamma_i Phi_ci and the partial sum of squares.
+//     few tokens must still spread over many SMs); CTA (blk, part) forms
+//     Phi * gamma over its part once in shared memory and every warp streams
+//     4 tokens of that part with float4 loads, so each value read is used 4
+//     times; the sums run as packed fp32x2 FMAs over column pairs.  It writes,
+//     per token and part, the 8 partial projections sum_i s_i gamma_i Phi_ci
+//     and the partial sum of squares.
 // (B) mhc_read: one warp per token folds the two halves into
 //     l = (sum / r), r = sqrt(sum of squares / 2H + eps), forms H_pre, H_post
 //     and H_res = Sinkhorn(exp(l[4:8])), then reads x = H_pre0 s_0 + H_pre1 s_1
 //     and writes RMSNorm(x) * gain.  The stream rows are read twice (sum of
 //     squares, then the write), the second time from L1/L2.
 // ---------------------------------------------------------------------------
-constexpr int MHCA_WARPS = 8, MHCA_TOK = 8;  // tokens per warp
+constexpr int MHCA_WARPS = 12, MHCA_TOK = 4;  // tokens per warp
 constexpr int MHCA_THREADS = MHCA_WARPS * 32;
 constexpr int MHCB_WARPS = 8;
 
@@ -245,12 +246,14 @@ __global__ void __launch_bounds__(MHCA_THREADS, 1)
   const int D = 2 * H, PL = D / parts, PL4 = PL / 4;
   const int i0 = p * PL;                  // this part's first entry of the flattened streams
   const int stream = i0 / H, col0 = i0 % H;  // a part lies inside one stream
-  float4* sphi = sm4;             // [8][PL4]
-  float4* sgam = sm4 + 8 * PL4;   // [PL4]
+  float4* sw = sm4;  // [8][PL4]: Phi * gamma over this part, formed once per CTA
   for (int i = threadIdx.x; i < PL4; i += MHCA_THREADS) {
+    const float4 g = reinterpret_cast<const float4*>(gamma + i0)[i];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) sphi[c * PL4 + i] = reinterpret_cast<const float4*>(phi + (int64_t)c * D + i0)[i];
-    sgam[i] = reinterpret_cast<const float4*>(gamma + i0)[i];
+    for (int c = 0; c < 8; ++c) {
+      const float4 ph = reinterpret_cast<const float4*>(phi + (int64_t)c * D + i0)[i];
+      sw[c * PL4 + i] = make_float4(ph.x * g.x, ph.y * g.y, ph.z * g.z, ph.w * g.w);
+    }
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -259,32 +262,38 @@ __global__ void __launch_bounds__(MHCA_THREADS, 1)
   const int ntok = (int)(T - t0 < MHCA_TOK ? T - t0 : MHCA_TOK);
   const int H4 = H / 4;
   const float4* base = reinterpret_cast<const float4*>(s + ((int64_t)stream * T + t0) * H + col0);
-  float acc[MHCA_TOK][9];
+  // per token: 8 projections and the sum of squares, each as a pair of
+  // partial sums (even and odd columns) so the products run as packed fp32x2 FMAs
+  float2 acc[MHCA_TOK][9];
 #pragma unroll
   for (int j = 0; j < MHCA_TOK; ++j)
 #pragma unroll
-    for (int c = 0; c < 9; ++c) acc[j][c] = 0.f;
+    for (int c = 0; c < 9; ++c) acc[j][c] = make_float2(0.f, 0.f);
 #pragma unroll 2
   for (int f = lane; f < PL4; f += 32) {
     float4 v[MHCA_TOK];
 #pragma unroll
     for (int j = 0; j < MHCA_TOK; ++j) v[j] = j < ntok ? __ldcs(base + (int64_t)j * H4 + f) : make_float4(0, 0, 0, 0);
-    const float4 g = sgam[f];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      const float4 ph = sphi[c * PL4 + f];
-      const float4 w = make_float4(ph.x * g.x, ph.y * g.y, ph.z * g.z, ph.w * g.w);
+      const float4 w = sw[c * PL4 + f];
 #pragma unroll
-      for (int j = 0; j < MHCA_TOK; ++j) acc[j][c] += v[j].x * w.x + v[j].y * w.y + v[j].z * w.z + v[j].w * w.w;
+      for (int j = 0; j < MHCA_TOK; ++j) {
+        acc[j][c] = ffma2(make_float2(v[j].x, v[j].y), make_float2(w.x, w.y), acc[j][c]);
+        acc[j][c] = ffma2(make_float2(v[j].z, v[j].w), make_float2(w.z, w.w), acc[j][c]);
+      }
     }
 #pragma unroll
-    for (int j = 0; j < MHCA_TOK; ++j) acc[j][8] += v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
+    for (int j = 0; j < MHCA_TOK; ++j) {
+      acc[j][8] = ffma2(make_float2(v[j].x, v[j].y), make_float2(v[j].x, v[j].y), acc[j][8]);
+      acc[j][8] = ffma2(make_float2(v[j].z, v[j].w), make_float2(v[j].z, v[j].w), acc[j][8]);
+    }
   }
 #pragma unroll
   for (int j = 0; j < MHCA_TOK; ++j)
 #pragma unroll
     for (int c = 0; c < 9; ++c) {
-      const float r = warp_sum(acc[j][c]);
+      const float r = warp_sum(acc[j][c].x + acc[j][c].y);
       if (lane == c && j < ntok) part[((t0 + j) * parts + p) * 9 + c] = r;
     }
 }
@@ -526,7 +535,7 @@ cudaError_t launch_mhc_token(const float* s, int64_t T, int H, const float* gamm
   return cudaGetLastError();
 }
 
-size_t mhc_partial_smem(int H) { return (size_t)9 * H * sizeof(float); }
+size_t mhc_partial_smem(int H) { return (size_t)8 * H * sizeof(float); }  // Phi * gamma of half the streams
 
 cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf,
