@@ -119,9 +119,64 @@ __global__ void rmsnorm_kernel(const float* x, int H, int64_t step, int64_t off,
   const float inv = rsqrtf(ss / H + eps);
   for (int i = threadIdx.x; i < H; i += blockDim.x) y[r * H + i] = from_f<T>(xr[i] * inv * gain[i]);
 }
+// The same for H = 512 NPL: 128 threads keep the row's NPL float4 each in
+// registers (one pass over the row), one block reduction, vector stores.
+template <typename T, int NPL>
+__global__ void __launch_bounds__(128)
+    rmsnorm_vec_kernel(const float* __restrict__ x, int64_t step, int64_t off, const float* __restrict__ gain,
+                       float eps, T* __restrict__ y) {
+  constexpr int H = 512 * NPL;
+  __shared__ float red[4];
+  griddep_launch_dependents();  // a decode GEMM after this may start streaming its weights
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t r = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + (r * step + off) * H);
+  float4 a[NPL];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    a[i] = xr[tid + 128 * i];
+    ss += a[i].x * a[i].x + a[i].y * a[i].y + a[i].z * a[i].z + a[i].w * a[i].w;
+  }
+  ss = warp_sum(ss);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  const float inv = rsqrtf((red[0] + red[1] + red[2] + red[3]) / H + eps);
+  const float4* g4 = reinterpret_cast<const float4*>(gain);
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const float4 g = g4[tid + 128 * i];
+    const float x0 = a[i].x * inv * g.x, x1 = a[i].y * inv * g.y, x2 = a[i].z * inv * g.z, x3 = a[i].w * inv * g.w;
+    if constexpr (sizeof(T) == 2) {
+      uint2 u;
+      u.x = pack_bf16x2(x0, x1);
+      u.y = pack_bf16x2(x2, x3);
+      reinterpret_cast<uint2*>(y + r * H)[tid + 128 * i] = u;
+    } else {
+      reinterpret_cast<float4*>(y + r * H)[tid + 128 * i] = make_float4(x0, x1, x2, x3);
+    }
+  }
+}
+
 cudaError_t launch_rmsnorm(const float* x, int64_t rows, int H, int64_t step, int64_t off, const float* gain,
                            float eps, void* y, bool bf, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
+  if (H % 512 == 0) {
+#define LOOP_RMS(NPL)                                                                                          \
+  case NPL:                                                                                                    \
+    if (bf) rmsnorm_vec_kernel<bf16, NPL><<<(unsigned)rows, 128, 0, st>>>(x, step, off, gain, eps, (bf16*)y);   \
+    else rmsnorm_vec_kernel<float, NPL><<<(unsigned)rows, 128, 0, st>>>(x, step, off, gain, eps, (float*)y);    \
+    return cudaGetLastError();
+    switch (H / 512) {
+      LOOP_RMS(1)
+      LOOP_RMS(2)
+      LOOP_RMS(4)
+      LOOP_RMS(8)
+      LOOP_RMS(12)
+      default: break;
+    }
+#undef LOOP_RMS
+  }
   if (bf) rmsnorm_kernel<bf16><<<(unsigned)rows, 256, 0, st>>>(x, H, step, off, gain, eps, (bf16*)y);
   else rmsnorm_kernel<float><<<(unsigned)rows, 256, 0, st>>>(x, H, step, off, gain, eps, (float*)y);
   return cudaGetLastError();
