@@ -47,26 +47,6 @@ constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, D, true);
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
-// 2^x on the FMA pipe for both lanes of x (x <= 64): x = n + f with n the
-// nearest integer (1.5 * 2^23 added and removed) and f in [-1/2, 1/2], 2^f by
-// a cubic, and n added to the exponent bits.  The cubic's coefficients are the
-// minimax fit that exp2_poly_fit.py computes; relative error < 7.5e-5.  Inputs
-// below -125 give 2^-125, not 0, so masked scores never take this path.
-constexpr float P2_C0 = 0.9999280571937561f, P2_C1 = 0.6932609677314758f, P2_C2 = 0.2426111251115799f,
-                P2_C3 = 0.0551716685295105f;
-LOOP_DEV float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = fadd2(x, make_float2(12582912.f, 12582912.f));
-  const float2 n = fadd2(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
-  float2 p = ffma2(make_float2(P2_C3, P2_C3), f, make_float2(P2_C2, P2_C2));
-  p = ffma2(p, f, make_float2(P2_C1, P2_C1));
-  p = ffma2(p, f, make_float2(P2_C0, P2_C0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
 LOOP_DEV float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -74,18 +54,15 @@ LOOP_DEV float max3f(float a, float b, float c) {
 }
 
 // P for the 64 keys of one row: p = 2^(s scale - m_ref) as bf16 pairs into
-// pk, their sum added to rs2.  With POLY one pair in three is evaluated on the
-// FMA pipe so the MUFU unit is not the limit.
-template <bool POLY>
+// pk, their sum added to rs2.  The exponent argument is one packed fp32x2
+// FMA, the power of two ex2.approx on the MUFU unit (evaluating part of them
+// as a polynomial on the FMA pipe measured slower here: with one MMA issuer
+// per query tile the softmax is not MUFU-bound).
 LOOP_DEV void softmax_row(const float (&sv)[BKV], float2 sc, float2 nm, float (&pk)[32], float2& rs2) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const float2 xx = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sc, nm);
-    float2 pp;
-    if (POLY && (i % 3) == 1)
-      pp = exp2_poly2(xx);
-    else
-      pp = make_float2(ex2(xx.x), ex2(xx.y));
+    const float2 pp = make_float2(ex2(xx.x), ex2(xx.y));
     rs2 = fadd2(rs2, pp);
     pk[i] = __uint_as_float(pack_bf16x2(pp.x, pp.y));
   }
@@ -269,10 +246,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       float2 rs2 = make_float2(0.f, 0.f);
       {
         float pk[32];
-        if (masked)
-          softmax_row<false>(sv, sc, nm, pk, rs2);
-        else
-          softmax_row<true>(sv, sc, nm, pk, rs2);
+        softmax_row(sv, sc, nm, pk, rs2);
         tmem_st32(t_s, pk);
       }
       l = l * corr + (rs2.x + rs2.y);
