@@ -61,6 +61,10 @@ struct EpiP {
   const int32_t* table;  // QKV_FULL: KV page table (the call's first sequence) and its row stride
   int pps;
   float eps;
+  // MHC_WRITE: the next mHC site's Phi * gamma [8][2N], and where the
+  // partial projections of the new streams go, [M][2 N / BN][9] (NULL: none)
+  const float* pphig;
+  float* ppart;
 };
 
 LOOP_DEV void ld_chunk(uint32_t taddr, float (&v)[32]) {
@@ -123,6 +127,35 @@ LOOP_DEV void head_store_rope(uint32_t t0, bf16* dst, const float2* cs_row, bool
   }
 }
 
+// r[k] holds this lane's part of a sum for row group k (k = 0..7); the 8 lanes
+// whose low 3 bits are 0..7 and whose other bits agree hold the other parts.
+// Returns the total for row group (lane & 7), reduced in a fixed tree.
+LOOP_DEV float reduce_scatter8(const float (&r)[8], int lane) {
+  const bool b2 = lane & 4, b1 = lane & 2, b0 = lane & 1;
+  float t[4], u[2];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float keep = b2 ? r[k + 4] : r[k], give = b2 ? r[k] : r[k + 4];
+    t[k] = keep + __shfl_xor_sync(0xffffffffu, give, 4);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float keep = b1 ? t[k + 2] : t[k], give = b1 ? t[k] : t[k + 2];
+    u[k] = keep + __shfl_xor_sync(0xffffffffu, give, 2);
+  }
+  const float keep = b0 ? u[1] : u[0], give = b0 ? u[0] : u[1];
+  return keep + __shfl_xor_sync(0xffffffffu, give, 1);
+}
+
+// a . w0 + b . w1 over the 8 entries, as packed fp32x2 FMAs
+LOOP_DEV float dot8(float4 a, float4 b, float4 w0, float4 w1) {
+  float2 s = ffma2(make_float2(a.x, a.y), make_float2(w0.x, w0.y), make_float2(0.f, 0.f));
+  s = ffma2(make_float2(a.z, a.w), make_float2(w0.z, w0.w), s);
+  s = ffma2(make_float2(b.x, b.y), make_float2(w1.x, w1.y), s);
+  s = ffma2(make_float2(b.z, b.w), make_float2(w1.z, w1.w), s);
+  return s.x + s.y;
+}
+
 // tcgen05.ld / wait::ld are warp-collective: every lane of the warp executes
 // them in lockstep, and only the memory accesses of rows >= M are skipped.
 // Two epilogue warpgroups share a tile: `half` 0 takes the first 128
@@ -158,6 +191,12 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, int half, const EpiP
     const int row0 = row - lane;  // the warp's first row
     float4* xs4 = reinterpret_cast<float4*>(xs);
     const int64_t plane = (int64_t)p.M * p.N;
+    // next-site projections: this lane ends with the 9 sums of row 4 (lane & 7)
+    // + (lane >> 3) over the warp's 128 columns of both streams
+    const bool proj = MODE == Epi::MHC_WRITE && p.pphig != nullptr;
+    float pacc[9];
+#pragma unroll
+    for (int j = 0; j < 9; ++j) pacc[j] = 0.f;
 #pragma unroll 1
     for (int c = 4 * half; c < 4 * half + 4; ++c) {
       const int n = n0 + 32 * c;
@@ -181,6 +220,8 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, int half, const EpiP
             a[k] = __ldcs(reinterpret_cast<const float4*>(p.s + off));
             b[k] = __ldcs(reinterpret_cast<const float4*>(p.s + plane + off));
           }
+        } else {
+          a[k] = b[k] = make_float4(0.f, 0.f, 0.f, 0.f);  // rows past M add nothing to the projections
         }
       }
 #pragma unroll
@@ -206,9 +247,35 @@ LOOP_DEV void epilogue_tile(uint32_t tacc, int row, int n0, int half, const EpiP
           z.w = c1.z * a[k].w + c1.w * b[k].w + c0.w * y[k].w;
           *reinterpret_cast<float4*>(p.s + off) = x;
           *reinterpret_cast<float4*>(p.s + plane + off) = z;
+          a[k] = x;  // kept for the next site's projections
+          b[k] = z;
+        }
+      }
+      if (proj) {
+        // sum_i u_i gamma_i Phi_ci over this chunk's 32 columns of both
+        // streams (c < 8), and sum_i u_i^2 (c = 8), for each of the lane's 8 rows
+        const int col = n + 4 * col4;
+#pragma unroll
+        for (int j = 0; j < 9; ++j) {
+          float r[8];
+          const float4 w0 = j < 8 ? __ldg(reinterpret_cast<const float4*>(p.pphig + (int64_t)j * 2 * p.N + col))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 w1 = j < 8 ? __ldg(reinterpret_cast<const float4*>(p.pphig + (int64_t)j * 2 * p.N + p.N + col))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) r[k] = j < 8 ? dot8(a[k], b[k], w0, w1) : dot8(a[k], b[k], a[k], b[k]);
+          pacc[j] += reduce_scatter8(r, lane);
         }
       }
       __syncwarp();  // the tile is rewritten by the next chunk
+    }
+    if (proj) {
+      const int prow = row0 + 4 * (lane & 7) + (lane >> 3);
+      if (prow < p.M) {
+        float* dst = p.ppart + ((int64_t)prow * (2 * p.N / BN) + 2 * (n0 / BN) + half) * 9;
+#pragma unroll
+        for (int j = 0; j < 9; ++j) dst[j] = pacc[j];
+      }
     }
   } else if constexpr (MODE == Epi::SWIGLU) {
     const int F = p.N / 2;
@@ -671,6 +738,8 @@ cudaError_t launch_gemm_tc(const void* A, const void* W, int64_t M, int64_t N, i
   p.table = e.table;
   p.pps = e.pps;
   p.eps = e.eps;
+  p.pphig = e.next_phig;
+  p.ppart = e.part;
   switch (e.mode) {
     case Epi::F32: return launch_mode<Epi::F32>(ma, mb, (int)M, (int)N, (int)K, p, st);
     case Epi::RESID: return launch_mode<Epi::RESID>(ma, mb, (int)M, (int)N, (int)K, p, st);

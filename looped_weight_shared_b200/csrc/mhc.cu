@@ -592,6 +592,26 @@ cudaError_t launch_mhc_token(const float* s, int64_t T, int H, const float* gamm
 
 size_t mhc_partial_smem(int H) { return (size_t)8 * H * sizeof(float); }  // Phi * gamma of half the streams
 
+__global__ void mhc_phig_kernel(const float* __restrict__ gamma, const float* __restrict__ phi, int64_t D,
+                                float* __restrict__ out) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < 8 * D; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = phi[i] * gamma[i % D];
+}
+cudaError_t launch_mhc_phig(const float* gamma, const float* phi, int64_t D, float* out, cudaStream_t st) {
+  mhc_phig_kernel<<<(unsigned)std::min<int64_t>((8 * D + 255) / 256, 1024), 256, 0, st>>>(gamma, phi, D, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mhc_coef_read(const float* part, int parts, const float* s, int64_t T, int H, const float* gain,
+                                 int iters, float eps, float* coef, void* xh, bool bf, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (H != 4096 || parts < 1) return cudaErrorInvalidValue;
+  mhc_coef_kernel<<<(unsigned)((T + 127) / 128), 128, 0, st>>>(part, parts, T, 2 * H, iters, eps, coef);
+  if (bf) mhc_read1_kernel<bf16, 8><<<(unsigned)T, 128, 0, st>>>(s, T, coef, gain, eps, (bf16*)xh);
+  else mhc_read1_kernel<float, 8><<<(unsigned)T, 128, 0, st>>>(s, T, coef, gain, eps, (float*)xh);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* gamma, const float* phi,
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf,
                                 float* part, cudaStream_t st, int parts, bool fused_read) {

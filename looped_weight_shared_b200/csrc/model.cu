@@ -291,6 +291,10 @@ int32_t create_impl(const loop_config* cfg, const float* const* hw, uint64_t see
     LOOP_ALLOC(m.sites[s].phi, float*, 8 * 2 * H * 4);
     LOOP_RC(fill_f32(m, hw, seed, wi, 0, m.sites[s].gamma, 2 * H, true));
     LOOP_RC(fill_f32(m, hw, seed, wi + 1, site_stream(s), m.sites[s].phi, 16 * H, false));
+    if (bf && m.use_tc && H == 4096) {  // the prefill forms this site's projections in a GEMM epilogue
+      LOOP_ALLOC(m.sites[s].phig, float*, 8 * 2 * H * 4);
+      LOOP_CU(launch_mhc_phig(m.sites[s].gamma, m.sites[s].phi, 2 * H, m.sites[s].phig, 0));
+    }
   }
   // KV cache: one page pool per full-attention execution and one page table
   // per sequence shared by all of them (every execution of a sequence holds
@@ -333,6 +337,7 @@ int32_t create_impl(const loop_config* cfg, const float* const* hw, uint64_t see
   LOOP_ALLOC(w.xh, void*, T * H * es);
   LOOP_ALLOC(w.coef, float*, T * 8 * 4);
   w.mhc_part_floats = std::max<int64_t>(T * 18, 512 * 16 * 9);
+  if (H % 256 == 0) w.mhc_part_floats = std::max<int64_t>(w.mhc_part_floats, T * (2 * H / 256) * 9);
   LOOP_ALLOC(w.mhc_part, float*, w.mhc_part_floats * 4);
   if (m.use_tc && H % 64 == 0) {  // decode GEMM partials: up to 32 splits x 64 tokens x the widest projection
     int64_t maxn = std::max<int64_t>(2 * F, H);
@@ -492,6 +497,7 @@ cudaError_t project(Model& m, const void* A, const void* W, int64_t M, int64_t N
                     cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const double flops = 2.0 * (double)M * (double)N * (double)K;
+  m.w.part_formed = false;
   if (m.decoding && m.use_tc && m.w.cpart && gemm_skinny_supported(M, N, K)) {
     // decode: weight-streaming split-K GEMM, then the epilogue over the partials
     // (prefills never take it, so a prefill row is computed the same way
@@ -507,8 +513,11 @@ cudaError_t project(Model& m, const void* A, const void* W, int64_t M, int64_t N
     return timed(m, LOOP_K_OTHER, 0.0, 1, st,
                  [&] { return launch_epilogue_unfused(P, N, M, N, e, bf16_model(m), st, splits); });
   }
-  if (m.use_tc && gemm_tc_supported(M, N, K, e))
-    return timed(m, LOOP_K_GEMM, flops, 1, st, [&] { return launch_gemm_tc(A, W, M, N, K, e, st); });
+  if (m.use_tc && gemm_tc_supported(M, N, K, e)) {
+    const cudaError_t err = timed(m, LOOP_K_GEMM, flops, 1, st, [&] { return launch_gemm_tc(A, W, M, N, K, e, st); });
+    m.w.part_formed = err == cudaSuccess && e.mode == Epi::MHC_WRITE && e.part != nullptr;
+    return err;
+  }
   float* C = e.mode == Epi::F32 ? e.c : m.w.cbuf;
   const int64_t ldc = e.mode == Epi::F32 ? e.ldc : N;
   cudaError_t err = timed(m, LOOP_K_GEMM, flops, 1, st,
@@ -639,6 +648,11 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
   else LOOP_CU(cudaMemcpyAsync(w.h, hidden, T * H * 4, cudaMemcpyDeviceToDevice, st));
   const int first_block = c.n_prelude, last_block = c.n_prelude + c.n_block * c.n_loops - 1;
   float* s_buf = w.s;  // streams [2][T][H]
+  // A prefill's mHC-write projections also form the next site's partial
+  // projections (hidden 4096, tensor-core path), so that site reads its
+  // streams once instead of twice.
+  const bool fuse_sites = !m.decoding && bf && m.use_tc && H == 4096;
+  bool part_ready = false;  // w.mhc_part holds the current streams' partials for this site
   for (int e = 0; e < m.n_exec; ++e) {
     const int32_t* row = &m.table[5 * e];
     const int phys = row[0], kind = row[2], slot = row[3], region = row[4];
@@ -654,6 +668,11 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
           LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), 1, st, [&] {
             return launch_mhc_token(s_buf, T, (int)H, site.gamma, site.phi, gain, c.sinkhorn_iters, c.norm_eps,
                                     w.coef, w.xh, bf, st);
+          }));
+        } else if (part_ready) {  // partials formed by the projection that wrote the streams
+          LOOP_CU(timed(m, LOOP_K_MHC, (double)T * (8.0 * H + es * H + 32.0), 2, st, [&] {
+            return launch_mhc_coef_read(w.mhc_part, (int)(2 * H / 256), s_buf, T, (int)H, gain, c.sinkhorn_iters,
+                                        c.norm_eps, w.coef, w.xh, bf, st);
           }));
         } else {
           // decode at other widths: cut Phi into 16 parts so the partial kernel spreads over the
@@ -671,11 +690,20 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
         LOOP_CU(timed(m, LOOP_K_NORM, (double)T * H * (4 + es), 1, st,
                       [&] { return launch_rmsnorm(w.h, T, (int)H, 1, 0, gain, c.norm_eps, w.xh, bf, st); }));
       }
+      part_ready = false;
       EpiArgs out_epi;
       if (in_block) {
         out_epi.mode = Epi::MHC_WRITE;
         out_epi.s = s_buf;
         out_epi.coef = w.coef;
+        // the loop region's next site (none after its last write)
+        const SiteW* next = nullptr;
+        if (sub == 0) next = &m.sites[2 * (phys - c.n_prelude) + 1];
+        else if (e < last_block) next = &m.sites[2 * (m.table[5 * (e + 1)] - c.n_prelude)];
+        if (fuse_sites && next && next->phig) {
+          out_epi.next_phig = next->phig;
+          out_epi.part = w.mhc_part;
+        }
       } else {
         out_epi.mode = Epi::RESID;
         out_epi.c = w.h;
@@ -706,12 +734,14 @@ int32_t forward(Model& m, const int32_t* tokens, const float* hidden, int b0, in
             if (cp.exec == e && b0 == 0) LOOP_CU(capture(m, cp, false, nullptr, nullptr, S, st));
         }
         LOOP_CU(project(m, w.o, L.w_o, T, H, L.n_o_in, out_epi, st));
+        part_ready = out_epi.part != nullptr && w.part_formed;
       } else {
         EpiArgs ge;
         ge.mode = Epi::SWIGLU;
         ge.a = w.a;
         LOOP_CU(project(m, w.xh, L.w_gu, T, 2 * F, H, ge, st));
         LOOP_CU(project(m, w.a, L.w_down, T, H, F, out_epi, st));
+        part_ready = out_epi.part != nullptr && w.part_formed;
       }
     }
     if (e == last_block)

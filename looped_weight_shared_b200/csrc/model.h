@@ -57,6 +57,11 @@ struct EpiArgs {
   int pps = 0;                     // QKV_FULL: pages per sequence (table row stride)
   int n_lin = 0;
   float eps = 1e-6f;
+  // MHC_WRITE on the tensor-core path: also the next mHC site's partial
+  // projections of the new streams (next_phig = that site's Phi * gamma,
+  // [8][2H]), written to part [M][2 N / 256][9]; NULL: none
+  const float* next_phig = nullptr;
+  float* part = nullptr;
 };
 
 struct LayerW {
@@ -73,6 +78,7 @@ struct LayerW {
 struct SiteW {
   float* gamma = nullptr;  // [2H]
   float* phi = nullptr;    // [8][2H]
+  float* phig = nullptr;   // [8][2H] Phi * gamma entry by entry (for projections formed in a GEMM epilogue)
 };
 
 struct Work {
@@ -92,6 +98,7 @@ struct Work {
   int32_t* zeros = nullptr; // start positions of a prefill (all 0)
   float* mhc_part = nullptr;  // [T][parts][9] partial projections of the mHC prologue
   int64_t mhc_part_floats = 0;
+  bool part_formed = false;   // the last projection also wrote the next site's partials into mhc_part
   float* cpart = nullptr;     // split-K partial sums of the decode GEMM [32][64][max N]
   int64_t cpart_floats = 0;
   float* dec_attn = nullptr;  // decode attention chunk partials [B][n_q][ctx / 128][130]
@@ -191,6 +198,13 @@ cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* g
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf16,
                                 float* part, cudaStream_t st, int parts = 2, bool fused_read = false);
 size_t mhc_partial_smem(int H);
+// hidden 4096, the partial projections already formed ([T][parts][9], summed
+// in part order, e.g. by the mHC-write epilogue of the projection before):
+// the coefficient kernel and the one-pass reader
+// out[c][i] = phi[c][i] * gamma[i], c < 8, i < D
+cudaError_t launch_mhc_phig(const float* gamma, const float* phi, int64_t D, float* out, cudaStream_t st);
+cudaError_t launch_mhc_coef_read(const float* part, int parts, const float* s, int64_t T, int H, const float* gain,
+                                 int iters, float eps, float* coef, void* xh, bool bf16, cudaStream_t st);
 // one launch per site for a few tokens (decode), hidden 4096
 bool mhc_token_supported(int H);
 cudaError_t launch_mhc_token(const float* s, int64_t T, int H, const float* gamma, const float* phi,

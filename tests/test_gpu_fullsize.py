@@ -57,8 +57,10 @@ def _check_linear_capture(cap, state_gpu, nh=2, d=128):
         o_ref, st_ref = oracle.gla_recurrent(_np(cap["lq"][h]), _np(cap["lk"][h]), _np(cap["lv"][h]), g)
         got = o_gpu[:, h * d:(h + 1) * d]
         e, c = rel_err(got, o_ref), cosine(got, o_ref)
+        print(f"linear output head {h}: rel {e:.3g} cos {c:.6f}")
         assert e < TOL_BF16 and c > COS_BF16, ("linear output", h, e, c)
         e, c = rel_err(state_gpu[h], st_ref), cosine(state_gpu[h], st_ref)
+        print(f"linear state head {h}: rel {e:.3g} cos {c:.6f}")
         assert e < TOL_BF16 and c > COS_BF16, ("linear state", h, e, c)
 
 
@@ -71,6 +73,7 @@ def _check_full_capture(cap, S):
     got = np.stack([o[p] for p in rows])
     ref = np.concatenate([oracle.attention_naive(q[p:p + 1], K[:p + 1], V[:p + 1], q0=p) for p in rows])
     e, c = rel_err(got, ref), cosine(got, ref)
+    print(f"attention rows: rel {e:.3g} cos {c:.6f}")
     assert e < TOL_BF16 and c > COS_BF16, ("attention rows", e, c)
 
 
