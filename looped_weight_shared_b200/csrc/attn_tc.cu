@@ -92,14 +92,17 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* pv_done = p_full + 4;    // [X]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
 
-  // Unpacked: CTA (query-tile pair, query head, sequence).  Packed (a few new
+  // Unpacked: CTA (query head, sequence, query-tile pair).  Packed (a few new
   // tokens per sequence, grp * S <= 128): CTA (kv head, sequence) whose one
   // tile holds the S queries of each of the grp query heads sharing that kv
   // head, row r = (head kvh * grp + r / S, query r % S): the heads' q rows are
   // adjacent in q, so one box loads them, and K/V are read once per kv head.
+  // CTAs start in block-index order (x fastest), so the query-tile pair is
+  // the slowest index and counts down: the longest pairs of every head run
+  // first and the shortest fill the tail.
   const int grp = nq / nkv;
   const int npair = (S + 2 * BQ - 1) / (2 * BQ);
-  const int q0 = packed ? 0 : 2 * BQ * (npair - 1 - (int)blockIdx.x);  // longest rows first
+  const int q0 = packed ? 0 : 2 * BQ * (npair - 1 - (int)blockIdx.x);
   const int b = blockIdx.z;
   const int kvh = packed ? (int)blockIdx.y : (int)blockIdx.y / grp;
   const int h = packed ? kvh * grp : (int)blockIdx.y;  // the (first) query head
@@ -250,10 +253,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_st32(t_s, pk);
       }
       l = l * corr + (rs2.x + rs2.y);
-      // rescale O once the product of the previous key tile is done
-      if (j >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
+      // pv_done is waited by parity, which is exact only while at most one
+      // product is pending.  At step j that holds: the issuer saw PV(j - 2)
+      // done before it issued S(j), and PV(j) needs this step's P.  So the
+      // product of the previous key tile is awaited here before O is
+      // rescaled, and always at the last key tile, so that the final wait
+      // below also has at most one pending (without it, PV(nt - 2) and
+      // PV(nt - 1) could both be pending there, a parity that matches a
+      // completed phase, and O would be read early).
+      const bool rescale = __any_sync(0xffffffffu, corr != 1.f);
+      if (j >= 1 && (rescale || j == nt[x] - 1)) {
         ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (j - 1) & 1, status, STATUS_WAIT_EPILOGUE));
         if (!ok) break;
+      }
+      if (j >= 1 && rescale) {
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
