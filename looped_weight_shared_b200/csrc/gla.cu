@@ -13,20 +13,21 @@
 // chunked form is exact for any chunk length), so every product is a full
 // M = 128 tensor-core tile.
 //
-// One CTA per (sequence, head) walks the tiles in order (12 warps):
+// One CTA per (sequence, head) walks the tiles in order (18 warps):
 //   warp 0      TMA producer: Q, K and V of the tile ([128][128] bf16 each,
 //               two 64-column boxes, 128-byte swizzle), each refilled as soon
 //               as the products that read it are done;
-//   warp 1      one thread issues the tcgen05.mma products:
+//   warp 1      allocates / frees the 512 TMEM columns; one thread issues
+//               the tcgen05.mma products:
 //                 P   = Q K^T                       (TMEM, fp32)
 //                 O_x = Q S_prev                    (S as bf16 hi + lo, MN-major)
 //                 R  += K^T V^                      (K read MN-major as A)
 //                 O_a = A V                         (A from TMEM, hi + lo)
 //               where R is the fp32 state, resident in TMEM for the whole
 //               sequence;
-//   warp 2      allocates / frees the 512 TMEM columns;
-//   warps 4-11  each owns one TMEM lane quarter (warp % 4) and one half of
-//               the 128 columns: the decayed scores A = P * D written back
+//   warps 2-17  each owns one TMEM lane quarter (warp % 4) and a quarter
+//               of the 128 columns (so each step of the per-tile chain below
+//               is split 16 ways): the decayed scores A = P * D written back
 //               over P as bf16 hi + lo (the A operand of O_a), V^ = diag(exp(
 //               b_last - b)) V as hi + lo in shared memory, the state step
 //               (R -> S_prev hi + lo in shared memory, R *= exp(b_last)), and
@@ -50,7 +51,7 @@ namespace {
 constexpr int DK = 128;
 constexpr int CT = 128;                       // tokens per tile
 constexpr int TILE = CT * 128 * 2;            // one [128][128] bf16 operand: two boxes [128][64]
-constexpr int THREADS = 384;
+constexpr int THREADS = 576;  // producer, MMA issuer + TMEM allocator, 16 epilogue warps
 constexpr int OFF_Q = 0, OFF_K = TILE, OFF_V = 2 * TILE, OFF_SHI = 3 * TILE, OFF_SLO = 4 * TILE,
               OFF_VHI = 5 * TILE, OFF_VLO = 6 * TILE, OFF_B2 = 7 * TILE;
 constexpr int NB2 = 3;                        // gate buffers (tiles t, t + 1 and one in flight)
@@ -122,10 +123,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBARS; ++i) mbar_init(&bar[i], i >= B_SR ? 8u : 1u);
+    for (int i = 0; i < NBARS; ++i) mbar_init(&bar[i], i >= B_SR ? 16u : 1u);
     fence_mbar_init();
   }
-  if (warp == 2) tmem_alloc(tmem_slot, 512);
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -202,10 +203,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         scores();
       }
     }
-  } else if (warp >= 4) {
-    const int ew = warp - 4;
+  } else if (warp >= 2) {
+    const int ew = warp - 2;
     const int quarter = warp & 3;     // TMEM lanes 32 quarter .. (fixed by the warp's rank)
-    const int cb = 64 * (ew >> 2);    // this warp's column half
+    const int cb = 32 * (ew >> 2);    // this warp's 32 columns
     const int r = 32 * quarter + lane;  // the row this thread owns: token t, key s or state row
     const uint32_t lo_lane = (uint32_t)(32 * quarter) << 16;
     const float* glh = gl + bh * S + t0;
@@ -247,9 +248,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       const float dl = ex2(b2s[(j % NB2) * CT + CT - 1]);
       const float* src = s_in ? s_in + r * 128 : nullptr;
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        const int col = cb + 32 * hh;
+{  // this thread's 32 columns
+        const int col = cb;
         float s[32];
         if (j == 0) {
 #pragma unroll
@@ -292,9 +292,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_DS], last & 1, status, STATUS_WAIT_EPILOGUE))) return false;
       tc_fence_after();
       float* dst = s_out + r * 128;
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        const int col = cb + 32 * hh;
+{  // this thread's 32 columns
+        const int col = cb;
         float s[32];
         tmem_ld32(tmem + T_R + lo_lane + col, s);
         tc_wait_ld();
@@ -311,7 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int valid = min(CT, Sl - j * CT);
       const float w = r < valid ? ex2(bb[CT - 1] - bb[r]) : 0.f;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int ch = 0; ch < 4; ++ch) {
         const uint32_t off = sw(r, cb / 8 + ch, CT);
         const uint4 u = *reinterpret_cast<const uint4*>(smem + OFF_V + off);
         const uint32_t in[4] = {u.x, u.y, u.z, u.w};
@@ -337,9 +336,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int valid = min(CT, Sl - j * CT);
       const float bt = bb[r];
       const bool row_ok = r < valid;
-#pragma unroll 1
-      for (int g = 0; g < 2; ++g) {
-        const int col = cb + 32 * g;
+{  // this thread's 32 keys
+        const int col = cb;
         float p[32];
         tmem_ld32(tmem + T_P + lo_lane + col, p);
         tc_wait_ld();
@@ -367,9 +365,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int c0 = c * CT, valid = min(CT, Sl - c0);
       const float et = ex2(b2s[(c % NB2) * CT + r]);
       bf16* dst = out + ((int64_t)b * S + t0 + c0 + r) * ((int64_t)nh * 128) + h * 128;
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        const int col = cb + 32 * hh;
+{  // this thread's 32 columns
+        const int col = cb;
         float x[32], a[32];
         tmem_ld32(tmem + T_OX + lo_lane + col, x);
         tmem_ld32(tmem + T_OA + lo_lane + col, a);
@@ -402,7 +399,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
