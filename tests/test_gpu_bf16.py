@@ -76,6 +76,34 @@ def test_group9b_bf16_matches_oracle(S):
         L.loop_model_destroy(g)
 
 
+def test_group9b_extend_matches_oracle():
+    """loop_extend at the 9B width: 6 new tokens on each of 2 sequences, all
+    positions, against the oracle's decode steps.  At hidden 4096 an append
+    runs the prefill kernels: the packed flash tile (4 query heads x 6 rows),
+    the chunked GLA continuing each state, and the next mHC site's partial
+    projections formed in the mHC-write epilogue."""
+    w = W.WORKLOADS["probe_decode_b64_ctx4096"]
+    B, S, k = 2, 40, 6
+    m = dict(w["model"], max_batch=B, max_ctx=S + k)
+    g = L.loop_model_create(L.make_config(**m), seed=9)
+    try:
+        o = oracle.Model(oracle.make_config(**m), seed=9)
+        tok = seeded.tokens(9, B, S, m["vocab"])
+        ext = seeded.tokens(9, B, k, m["vocab"], stream=seeded.S_DECODE_TOKENS)
+        o.prefill(tok)
+        out = torch.empty((B, m["vocab"]), device="cuda")
+        L.loop_prefill(g, tokens=torch.from_numpy(tok).cuda(), out=out)
+        got = torch.empty((B, k, m["vocab"]), device="cuda")
+        L.loop_extend(g, torch.from_numpy(ext).cuda(), got, flags=L.LOOP_ALL_POSITIONS)
+        torch.cuda.synchronize()
+        ref = np.stack([o.decode_step(ext[:, t]) for t in range(k)], axis=1)
+        check(got.cpu().numpy(), ref)
+        assert [L.loop_seq_len(g, b) for b in range(B)] == [S + k] * B
+        assert L.loop_device_status() == 0
+    finally:
+        L.loop_model_destroy(g)
+
+
 MID = dict(hidden=512, ffn=512, vocab=2048, n_q=4, n_kv=2, head_dim=128, n_lin=4, lin_dim=128, dtype=1)
 
 
