@@ -37,7 +37,7 @@ DEFAULT_WORKLOAD = "loop9b_prefill_b4_s8192"
 #   metrics, see profiles/launches_loop9b_prefill_b4_s8192.md)
 # - decode attention: 1.085 GB per launch on the probe_decode_b64_ctx4096
 #   workload (64 x 4096 keys), scaled by keys to 32,787
-GEMM_TRAFFIC_PER_LAUNCH = 3.32e9
+GEMM_TRAFFIC_PER_LAUNCH = 3.94e9
 DECODE_ATTN_TRAFFIC_PER_LAUNCH = 1.085e9 * 32787 / 4097
 LONG_WORKLOAD = "loop9b_prefill_b1_s262144"
 EXTEND_K = 8  # tokens per sequence of the timed loop_extend steps
