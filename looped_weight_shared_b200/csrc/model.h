@@ -198,11 +198,11 @@ cudaError_t launch_mhc_prologue(const float* s, int64_t T, int H, const float* g
                                 const float* gain, int iters, float eps, float* coef, void* xh, bool bf16,
                                 float* part, cudaStream_t st, int parts = 2, bool fused_read = false);
 size_t mhc_partial_smem(int H);
+// out[c][i] = phi[c][i] * gamma[i], c < 8, i < D
+cudaError_t launch_mhc_phig(const float* gamma, const float* phi, int64_t D, float* out, cudaStream_t st);
 // hidden 4096, the partial projections already formed ([T][parts][9], summed
 // in part order, e.g. by the mHC-write epilogue of the projection before):
 // the coefficient kernel and the one-pass reader
-// out[c][i] = phi[c][i] * gamma[i], c < 8, i < D
-cudaError_t launch_mhc_phig(const float* gamma, const float* phi, int64_t D, float* out, cudaStream_t st);
 cudaError_t launch_mhc_coef_read(const float* part, int parts, const float* s, int64_t T, int H, const float* gain,
                                  int iters, float eps, float* coef, void* xh, bool bf16, cudaStream_t st);
 // one launch per site for a few tokens (decode), hidden 4096
