@@ -92,17 +92,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* pv_done = p_full + 4;    // [X]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
 
-  // Unpacked: CTA (query head, sequence, query-tile pair).  Packed (a few new
+  // Unpacked: CTA (query-tile pair, query head, sequence).  Packed (a few new
   // tokens per sequence, grp * S <= 128): CTA (kv head, sequence) whose one
   // tile holds the S queries of each of the grp query heads sharing that kv
   // head, row r = (head kvh * grp + r / S, query r % S): the heads' q rows are
   // adjacent in q, so one box loads them, and K/V are read once per kv head.
-  // CTAs start in block-index order (x fastest), so the query-tile pair is
-  // the slowest index and counts down: the longest pairs of every head run
-  // first and the shortest fill the tail.
   const int grp = nq / nkv;
   const int npair = (S + 2 * BQ - 1) / (2 * BQ);
-  const int q0 = packed ? 0 : 2 * BQ * (npair - 1 - (int)blockIdx.x);
+  const int q0 = packed ? 0 : 2 * BQ * (npair - 1 - (int)blockIdx.x);  // a head's longest pairs first
   const int b = blockIdx.z;
   const int kvh = packed ? (int)blockIdx.y : (int)blockIdx.y / grp;
   const int h = packed ? kvh * grp : (int)blockIdx.y;  // the (first) query head
