@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       const float dl = ex2(b2s[(j % NB2) * CT + CT - 1]);
       const float* src = s_in ? s_in + r * 128 : nullptr;
-{  // this thread's 32 columns
+      {  // this thread's 32 columns
         const int col = cb;
         float s[32];
         if (j == 0) {
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&bar[B_DS], last & 1, status, STATUS_WAIT_EPILOGUE))) return false;
       tc_fence_after();
       float* dst = s_out + r * 128;
-{  // this thread's 32 columns
+      {  // this thread's 32 columns
         const int col = cb;
         float s[32];
         tmem_ld32(tmem + T_R + lo_lane + col, s);
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int valid = min(CT, Sl - j * CT);
       const float bt = bb[r];
       const bool row_ok = r < valid;
-{  // this thread's 32 keys
+      {  // this thread's 32 keys
         const int col = cb;
         float p[32];
         tmem_ld32(tmem + T_P + lo_lane + col, p);
@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int c0 = c * CT, valid = min(CT, Sl - c0);
       const float et = ex2(b2s[(c % NB2) * CT + r]);
       bf16* dst = out + ((int64_t)b * S + t0 + c0 + r) * ((int64_t)nh * 128) + h * 128;
-{  // this thread's 32 columns
+      {  // this thread's 32 columns
         const int col = cb;
         float x[32], a[32];
         tmem_ld32(tmem + T_OX + lo_lane + col, x);
